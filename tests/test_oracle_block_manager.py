@@ -1,0 +1,214 @@
+"""Pins for the oracle block manager (CPU only).
+
+Pinned to the pages' worked numbers (tests/golden/pages_worked_examples.json),
+to the invariants the pages state (a block is free exactly when no sequence
+holds it; freeing at refcount 0 returns the block; a shared page is copied only
+when written) and to brute-force enumeration on random operation sequences.
+"""
+
+import numpy as np
+import pytest
+
+import oracle
+from oracle import BlockManager, OutOfBlocks
+from paged_kv_cache_heads_b200 import workloads as W
+
+
+def check_invariants(bm: BlockManager):
+    """Free list and held blocks partition the pool; refcounts equal holder counts."""
+    free = list(bm.free)
+    assert len(set(free)) == len(free), "duplicate in free list"
+    holders = np.zeros(bm.num_blocks, dtype=np.int64)
+    for sid, row in bm.tables.items():
+        for b in row:
+            holders[b] += 1
+        assert len(row) == -(-bm.lens[sid] // bm.block_size)
+    assert list(holders) == list(bm.ref)
+    held = {b for b in range(bm.num_blocks) if bm.ref[b] > 0}
+    assert held.isdisjoint(free)
+    assert len(held) + len(free) == bm.num_blocks
+
+
+def test_short_generation_holds_only_its_pages(golden):
+    ex = golden["short_generation"]
+    bm = BlockManager(256, ex["block_size"])
+    bm.add_seq(1, ex["generated_tokens"])
+    assert len(bm.blocks_of(1)) == 4                       # ceil(50 / 16)
+    assert len(bm.blocks_of(1)) * ex["block_size"] < ex["preallocated_tokens"]
+    assert bm.num_free() == 256 - 4
+    check_invariants(bm)
+
+
+def test_128k_context_fills_8192_blocks_exactly(golden):
+    ex = golden["blocks_for_128k"]
+    bm = BlockManager(ex["stated_blocks"], ex["block_size"])
+    bm.add_seq(0, ex["context_tokens"])
+    assert bm.num_free() == 0 and len(bm.blocks_of(0)) == ex["stated_blocks"]
+    with pytest.raises(OutOfBlocks):
+        bm.append_tokens(0, 1)
+    assert bm.seq_len(0) == ex["context_tokens"]          # unchanged by the failed append
+    check_invariants(bm)
+
+
+def test_max_blocks_per_seq_caps_context(golden):
+    cfg = golden["default_config"]
+    bm = BlockManager(cfg["max_blocks_per_seq"] + 1, cfg["block_size"])
+    bm.add_seq(0, cfg["max_blocks_per_seq"] * cfg["block_size"])
+    table, lens = bm.block_table([0], cfg["max_blocks_per_seq"])
+    assert lens[0] == 8192 and (table >= 0).all()
+    bm.append_tokens(0, 1)
+    with pytest.raises(ValueError):
+        bm.block_table([0], cfg["max_blocks_per_seq"])
+
+
+def test_three_requests_share_prompt(golden):
+    ex = golden["three_requests"]
+    bs = 16
+    P, Q = ex["reading_system_prompt_tokens"], ex["reading_question_tokens"]
+    bm = BlockManager(512, bs)
+    bm.add_seq(100, P)                                     # the cached system prompt
+    bm.fork(100, 1, P)                                     # A
+    bm.fork(100, 2, P)                                     # B
+    bm.free_seq(100)
+    bm.append_tokens(1, Q + ex["A"]["generated"])
+    bm.append_tokens(2, Q + ex["B"]["generated"])
+    bm.add_seq(3, Q + ex["C"]["generated"])               # C: no system prompt
+    prompt_blocks = bm.blocks_of(1)[: P // bs]
+    assert prompt_blocks == bm.blocks_of(2)[: P // bs]
+    assert all(bm.refcount(b) == 2 for b in prompt_blocks)
+    assert set(bm.blocks_of(3)).isdisjoint(bm.blocks_of(1) + bm.blocks_of(2))
+    held_tokens = (512 - bm.num_free()) * bs
+    assert held_tokens < ex["stated_max_fraction"] * 3 * ex["preallocated_tokens_each"]
+    bm.free_seq(2)                                         # B finishes first
+    assert all(bm.refcount(b) == 1 for b in prompt_blocks)
+    assert not set(prompt_blocks) & set(bm.free)
+    check_invariants(bm)
+
+
+def test_free_at_refcount_zero_returns_blocks_in_order():
+    bm = BlockManager(10, 4, initial_free_order=[9, 8, 7, 6, 5, 4, 3, 2, 1, 0])
+    bm.add_seq(0, 10)                                      # blocks 9, 8, 7
+    bm.fork(0, 1, 6)                                       # shares 9, 8
+    bm.free_seq(0)
+    assert list(bm.free)[-1:] == [7]                       # only 7 reached refcount 0
+    assert bm.refcount(9) == 1 and bm.refcount(8) == 1
+    bm.free_seq(1)
+    assert list(bm.free)[-3:] == [7, 9, 8]
+    check_invariants(bm)
+
+
+def test_copy_on_write_only_for_shared_partial_block():
+    bm = BlockManager(20, 4, initial_free_order=list(range(20)))
+    bm.add_seq(0, 6)                                       # blocks 0, 1 (block 1 half full)
+    bm.fork(0, 1)
+    bm.fork(0, 2)
+    assert bm.refcount(1) == 3
+    slots, pairs = bm.append_tokens(1, 1)                 # shared partial block -> copy
+    assert pairs == [(1, 2)] and bm.blocks_of(1) == [0, 2] and slots == [2 * 4 + 2]
+    assert bm.refcount(1) == 2 and bm.refcount(2) == 1
+    slots, pairs = bm.append_tokens(1, 1)                 # now private: no copy
+    assert pairs == [] and slots == [2 * 4 + 3]
+    _, pairs = bm.append_tokens(2, 3)
+    assert pairs == [(1, 3)]
+    _, pairs = bm.append_tokens(0, 1)                     # last holder writes in place
+    assert pairs == [] and bm.blocks_of(0) == [0, 1]
+    check_invariants(bm)
+
+
+def test_block_aligned_share_needs_no_copy():
+    bm = BlockManager(10, 4)
+    bm.add_seq(0, 8)
+    bm.fork(0, 1)
+    _, pairs = bm.append_tokens(1, 5)
+    assert pairs == [] and bm.blocks_of(1)[:2] == bm.blocks_of(0)
+    check_invariants(bm)
+
+
+def test_failed_operations_change_nothing():
+    bm = BlockManager(5, 4)
+    bm.add_seq(0, 7)
+    bm.fork(0, 1)
+    before = (list(bm.free), list(bm.ref), {k: list(v) for k, v in bm.tables.items()}, dict(bm.lens))
+    with pytest.raises(OutOfBlocks):
+        bm.append_tokens(1, 14)                            # needs a copy + 3 new blocks, 3 free
+    with pytest.raises(OutOfBlocks):
+        bm.add_seq(2, 13)
+    with pytest.raises(ValueError):
+        bm.add_seq(0, 1)
+    with pytest.raises(ValueError):
+        bm.fork(0, 1)
+    with pytest.raises(ValueError):
+        bm.free_seq(7)
+    after = (list(bm.free), list(bm.ref), {k: list(v) for k, v in bm.tables.items()}, dict(bm.lens))
+    assert before == after
+
+
+def test_prefix_config_copy_count():
+    """48 sharers of a 1992-token prefix: 47 copies, the last sharer writes in place;
+    a 2000-token (block-aligned) prefix needs none."""
+    for P, expect in ((1992, 47), (2000, 0)):
+        wl = W.prefix_cow_decode(prefix_len=P)
+        bm = BlockManager(wl.geometry.num_blocks, 16, wl.initial_free_order)
+        n_pairs = 0
+        for op in wl.ops:
+            if op.kind == "add":
+                bm.add_seq(op.seq, op.n)
+            elif op.kind == "fork":
+                bm.fork(op.parent, op.seq, op.n)
+            elif op.kind == "append":
+                n_pairs += len(bm.append_tokens(op.seq, op.n)[1])
+        assert n_pairs == expect
+        check_invariants(bm)
+
+
+def test_slots_enumerate_sequence_blocks():
+    """Brute force: the slots of a sequence are exactly the slots of its blocks, in order."""
+    rng = np.random.default_rng(9)
+    bm = BlockManager(64, 8, initial_free_order=rng.permutation(64))
+    slots = bm.add_seq(0, 29)
+    expect = [b * 8 + o for b in bm.blocks_of(0) for o in range(8)][:29]
+    assert slots == expect
+    assert bm.slot_mapping(0, 5, 10) == expect[5:15]
+
+
+@pytest.mark.parametrize("seed", range(6))
+def test_random_operation_sequences_keep_invariants(seed):
+    rng = np.random.default_rng(100 + seed)
+    bs = int(rng.choice([4, 8, 16]))
+    nb = int(rng.integers(8, 80))
+    bm = BlockManager(nb, bs, initial_free_order=rng.permutation(nb))
+    live, next_id = [], 0
+    for _ in range(300):
+        r = rng.random()
+        try:
+            if r < 0.3 or not live:
+                bm.add_seq(next_id, int(rng.integers(0, 3 * bs)))
+                live.append(next_id)
+                next_id += 1
+            elif r < 0.45:
+                p = int(rng.choice(live))
+                bm.fork(p, next_id, int(rng.integers(0, bm.seq_len(p) + 1)))
+                live.append(next_id)
+                next_id += 1
+            elif r < 0.85:
+                s = int(rng.choice(live))
+                before = bm.blocks_of(s)
+                L0 = bm.seq_len(s)
+                n = int(rng.integers(0, 2 * bs))
+                slots, pairs = bm.append_tokens(s, n)
+                after = bm.blocks_of(s)
+                assert len(slots) == n and len(pairs) <= 1
+                for p_, sl in zip(range(L0, L0 + n), slots):
+                    assert sl == after[p_ // bs] * bs + p_ % bs
+                for old, new in pairs:
+                    assert old == before[-1] and after[len(before) - 1] == new
+            else:
+                s = int(rng.choice(live))
+                bm.free_seq(s)
+                live.remove(s)
+        except OutOfBlocks:
+            pass
+        check_invariants(bm)
+    for s in list(live):
+        bm.free_seq(s)
+    assert bm.num_free() == nb and sorted(bm.free) == list(range(nb))
