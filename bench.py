@@ -1,0 +1,445 @@
+#!/usr/bin/env python
+"""Benchmark of the paged KV-cache hot path on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--impl ours|reference]
+
+One step = one pass of the hot path over one batch: copy-on-write copies (if
+the step has any), the slot-mapped store of the step's new tokens, and
+attention over the block tables (decode split-K + merge, chunked-prefill rows
+when present). Default workload: the Llama-7B-shape decode batch (32
+sequences, 32 q = 32 kv heads, head_dim 128, bf16, 16-token blocks, context
+lengths U{128..2048}); its ~570 MB of K/V per step is larger than the 126 MB
+L2, so no flush is needed between steps.
+
+Prints ONE JSON line on rank 0. ``value`` is query tokens per second over all
+ranks (each rank runs its own independent batch: weak scaling, no data-path
+collective). ``e2e`` repeats the measurement through the same C-ABI calls
+with the step's inputs copied from pinned host memory and the output read
+back inside the timed region. ``roofline`` is for the attention call, the
+dominant launch. ``--impl reference`` times the CPU oracle instead.
+"""
+
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "paged decode-attn query-tokens/s and KV-read HBM GB/s (% of B200 peak)"
+UNIT = "query-tokens/s"
+
+# DRAM bytes per attention call from one ncu capture of this workload
+# (dram__bytes_read.sum + dram__bytes_write.sum, both attention kernels),
+# valid only while the kernel sources are byte-identical to the captured ones.
+NCU_TRAFFIC = {}
+
+
+def _sources_digest() -> str:
+    h = hashlib.sha256()
+    for f in ("decode.cu", "prefill.cu", "pa_common.cuh"):
+        with open(os.path.join(ROOT, "paged_kv_cache_heads_b200", "csrc", f), "rb") as fh:
+            h.update(fh.read())
+    return h.hexdigest()[:16]
+
+
+def measured_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        with open(path) as f:
+            d = json.load(f)
+        return float(d["hbm_gbs"]), float(d.get("bf16_tflops", 1590.0)), "measured"
+    return 6650.0, 1590.0, "fallback"
+
+
+# --------------------------------------------------------------------------
+# clocks sampled during the timed region
+# --------------------------------------------------------------------------
+
+class ClockSampler:
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.gpu = gpu_index
+        self.proc = None
+        self.lines = []
+
+    def __enter__(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.gpu), "--query-gpu=" + self.FIELDS, "--format=csv,noheader,nounits",
+                 "-lms", "100"], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            self._t = threading.Thread(target=self._read, daemon=True)
+            self._t.start()
+            time.sleep(0.3)
+        except (OSError, FileNotFoundError):
+            self.proc = None
+        return self
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append(line.strip())
+
+    def __exit__(self, *exc):
+        if self.proc:
+            time.sleep(0.2)
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+
+    def summary(self):
+        rows = []
+        for ln in self.lines:
+            p = [x.strip() for x in ln.split(",")]
+            if len(p) < 9:
+                continue
+            try:
+                rows.append(dict(sm=float(p[1]), smax=float(p[2]), power=float(p[3]),
+                                 hw=p[5], hwt=p[6], swt=p[7], cap=p[8]))
+            except ValueError:
+                continue
+        if not rows:
+            return None
+        reasons = set()
+        for r in rows:
+            for key, name in (("hw", "hw_slowdown"), ("hwt", "hw_thermal_slowdown"),
+                              ("swt", "sw_thermal_slowdown"), ("cap", "sw_power_cap")):
+                if r[key].lower() == "active":
+                    reasons.add(name)
+        loaded = [r["sm"] for r in rows if r["power"] > 200] or [r["sm"] for r in rows]
+        return {"sm_mhz": statistics.median(loaded), "sm_max_mhz": max(r["smax"] for r in rows),
+                "reasons": sorted(reasons), "samples": len(rows)}
+
+
+# --------------------------------------------------------------------------
+# distributed helpers (also exercised by the CPU gloo tests)
+# --------------------------------------------------------------------------
+
+def dist_env():
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    return world, rank, local
+
+
+def reduce_max(value: float, device=None) -> float:
+    """Max of a float over all ranks (identity without a process group)."""
+    import torch
+    import torch.distributed as dist
+    if not (dist.is_available() and dist.is_initialized()):
+        return value
+    t = torch.tensor([value], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def reduce_sum(value: float, device=None) -> float:
+    import torch
+    import torch.distributed as dist
+    if not (dist.is_available() and dist.is_initialized()):
+        return value
+    t = torch.tensor([value], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.SUM)
+    return float(t.item())
+
+
+def barrier():
+    import torch.distributed as dist
+    if dist.is_available() and dist.is_initialized():
+        dist.barrier()
+
+
+# --------------------------------------------------------------------------
+# algorithmic work of one step
+# --------------------------------------------------------------------------
+
+def step_work(wl, step_tokens: int, step_pairs: int):
+    """Algorithmic bytes / flops of one step, from the workload's sizes only."""
+    geo = wl.geometry
+    e = 2 if geo.dtype == "bf16" else 4
+    row = geo.num_kv_heads * geo.head_dim * e                 # one token's K (or V) row, all heads
+    lens = wl.notes["context_lens"]
+    attn_kv = attn_qo = prefill_flops = 0
+    for L, ql in zip(lens, wl.q_lens):
+        if ql == 0:
+            continue
+        attn_kv += 2 * L * row + 4 * ((L + geo.block_size - 1) // geo.block_size)
+        attn_qo += 2 * ql * geo.num_q_heads * geo.head_dim * e
+        if ql > 1:
+            pairs = sum(L - ql + j + 1 for j in range(ql))
+            prefill_flops += 4 * geo.head_dim * pairs * geo.num_q_heads
+    store = 2 * 2 * step_tokens * row + 4 * step_tokens
+    copy = 2 * 2 * step_pairs * geo.block_size * row
+    return dict(attn_bytes=attn_kv + attn_qo, attn_kv_bytes=attn_kv, store_bytes=store, copy_bytes=copy,
+                prefill_flops=prefill_flops)
+
+
+def launches_per_step(b) -> int:
+    from paged_kv_cache_heads_b200 import pa_attention_workspace_size
+    wl, geo = b.wl, b.wl.geometry
+    n = (1 if b.num_step_tokens else 0) + (1 if b.step_pairs.shape[0] else 0) + 1
+    if pa_attention_workspace_size(len(wl.batch_seqs), geo.num_q_heads, wl.max_query_len, b.max_context_len,
+                                   b.desc) > 0:
+        n += 1
+    if wl.max_query_len > 1:
+        n += 1
+    return n
+
+
+# --------------------------------------------------------------------------
+# the oracle, timed on the host cores
+# --------------------------------------------------------------------------
+
+def blas_threads() -> int:
+    try:
+        from threadpoolctl import threadpool_info
+        n = [int(p.get("num_threads", 1)) for p in threadpool_info()]
+        return max(n) if n else 1
+    except Exception:
+        return 1
+
+
+def oracle_setup(wl):
+    """Replay everything before the step on the oracle (untimed)."""
+    import oracle
+    from oracle import scenario as oscen
+    from paged_kv_cache_heads_b200 import workloads as W
+    geo = wl.geometry
+    kc, vc = W.sentinel_cache(geo), W.sentinel_cache(geo)
+    bm = oracle.BlockManager(geo.num_blocks, geo.block_size, wl.initial_free_order)
+    n_setup = len(wl.ops) - wl.step_ops
+
+    class _Head:
+        pass
+    head = _Head()
+    head.ops = wl.ops[:n_setup]
+    oscen.replay_ops(head, kc, vc, bm)
+    step = []
+    for op in wl.ops[n_setup:]:
+        if op.kind == "append":
+            slots, pairs = bm.append_tokens(op.seq, op.n)
+            step.append((op, np.asarray(slots, np.int64), pairs))
+        elif op.kind == "add":
+            step.append((op, np.asarray(bm.add_seq(op.seq, op.n), np.int64), []))
+    tables, lens = bm.block_table(wl.batch_seqs, geo.max_blocks_per_seq)
+    return kc, vc, step, tables, lens
+
+
+def oracle_step(wl, state):
+    import oracle
+    kc, vc, step, tables, lens = state
+    for op, slots, pairs in step:
+        oracle.copy_blocks(kc, vc, pairs)
+        oracle.store_kv(kc, vc, op.k, op.v, slots)
+    return oracle.paged_attention(wl.q, kc, vc, tables, lens, wl.query_start_loc(), wl.scale)
+
+
+def time_oracle(wl, budget_s: float = 12.0, min_steps: int = 1, max_steps: int | None = None):
+    state = oracle_setup(wl)
+    times = []
+    t_all = time.perf_counter()
+    while True:
+        t0 = time.perf_counter()
+        oracle_step(wl, state)
+        times.append(time.perf_counter() - t0)
+        if max_steps is not None and len(times) >= max_steps:
+            break
+        if len(times) >= min_steps and time.perf_counter() - t_all > budget_s:
+            break
+    mean = sum(times) / len(times)
+    return dict(value=wl.num_q_tokens / mean, unit=UNIT, cores=blas_threads(), kind="oracle",
+                sample="%d full steps of %s (store + attention, NumPy float64), %.2f s each"
+                       % (len(times), wl.name, mean)), times
+
+
+# --------------------------------------------------------------------------
+# our arm
+# --------------------------------------------------------------------------
+
+def measure_ours(wl, steps: int, warmup: int, device, gpu_index: int):
+    import torch
+    import paged_kv_cache_heads_b200 as P
+    from paged_kv_cache_heads_b200 import scenario as gs
+
+    P.load_library()
+    P.pa_read_device_flags(clear=True)
+    b = gs.prepare(wl, device)
+    stream = torch.cuda.current_stream(device)
+    for _ in range(max(warmup, 1)):
+        gs.run_step(b)
+    torch.cuda.synchronize(device)
+
+    # ---- device-resident inputs
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(steps)]
+    start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    barrier()
+    torch.cuda.synchronize(device)
+    with ClockSampler(gpu_index) as clocks:
+        start.record(stream)
+        for i in range(steps):
+            gs.run_step(b, attention=False)
+            ev[i][0].record(stream)
+            gs.run_attention(b)
+            ev[i][1].record(stream)
+        end.record(stream)
+        torch.cuda.synchronize(device)
+    barrier()
+    ms_total = start.elapsed_time(end)
+    attn_ms = [a.elapsed_time(z) for a, z in ev]
+
+    # ---- end to end: inputs from pinned host memory, output read back, same calls
+    host_in = [t.cpu().pin_memory() for t in (b.q, b.step_k, b.step_v, b.step_slots, b.step_pairs,
+                                              b.block_tables, b.context_lens, b.query_start_loc)]
+    dev_in = [b.q, b.step_k, b.step_v, b.step_slots, b.step_pairs, b.block_tables, b.context_lens,
+              b.query_start_loc]
+    host_out = torch.empty(b.out.shape, dtype=b.out.dtype).pin_memory()
+    h2d = sum(t.numel() * t.element_size() for t in host_in)
+    d2h = host_out.numel() * host_out.element_size()
+
+    def e2e_step():
+        for h, d in zip(host_in, dev_in):
+            if h.numel():
+                d.copy_(h, non_blocking=True)
+        gs.run_step(b)
+        host_out.copy_(b.out, non_blocking=True)
+
+    for _ in range(max(warmup, 1)):
+        e2e_step()
+    torch.cuda.synchronize(device)
+    barrier()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(steps):
+        e2e_step()
+    e1.record(stream)
+    torch.cuda.synchronize(device)
+    barrier()
+    e2e_ms = e0.elapsed_time(e1)
+    flags = P.pa_read_device_flags(clear=True)
+    return dict(ms_total=ms_total, attn_ms=attn_ms, e2e_ms=e2e_ms, h2d=h2d, d2h=d2h, clocks=clocks.summary(),
+                launches=launches_per_step(b) * steps, step_tokens=b.num_step_tokens,
+                step_pairs=int(b.step_pairs.shape[0]), flags=flags, max_context_len=b.max_context_len)
+
+
+def workload_config(wl, world: int, l2_note: str):
+    geo = wl.geometry
+    lens = wl.notes["context_lens"]
+    return {"workload": wl.name, "num_seqs": len(wl.batch_seqs), "num_q_tokens": wl.num_q_tokens,
+            "num_q_heads": geo.num_q_heads, "num_kv_heads": geo.num_kv_heads, "head_dim": geo.head_dim,
+            "block_size": geo.block_size, "num_blocks": geo.num_blocks, "kv_dtype": geo.dtype,
+            "context_tokens": int(sum(lens)), "max_context_len": int(max(lens)),
+            "parallelism": "dp%d (independent replicas)" % world, "l2": l2_note}
+
+
+def build_workload(name: str):
+    from paged_kv_cache_heads_b200 import workloads as W
+    if name == "prefix_cow_p2000":
+        return W.prefix_cow_decode(prefix_len=2000)
+    return W.CONFIGS[name]()
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=50)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--workload", default="llama7b")
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    world, rank, local = dist_env()
+    hbm_peak, bf16_peak, peak_src = measured_peaks()
+
+    if args.impl == "reference":
+        if rank != 0:
+            return 0
+        wl = build_workload(args.workload)
+        budget = 60.0
+        cpu, times = time_oracle(wl, budget_s=budget, min_steps=args.steps + args.warmup,
+                                 max_steps=args.steps + args.warmup)
+        timed = times[args.warmup:] or times
+        ms = 1e3 * sum(timed) / len(timed)
+        value = wl.num_q_tokens / (ms / 1e3)
+        cpu["value"] = value
+        line = {"metric": METRIC, "value": value, "unit": UNIT, "n_gpus": args.gpus, "steps": len(timed),
+                "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
+                "vs_baseline": None, "dtype": "f64", "data": "synthetic (seeded)", "impl": "reference",
+                "config": workload_config(wl, 1, "host memory (CPU oracle)"), "cpu_baseline": cpu,
+                "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+                "gpu_launches": 0}
+        print(json.dumps(line), flush=True)
+        return 0
+
+    import torch
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device("cuda", local))
+    device = torch.device("cuda", local)
+    torch.cuda.set_device(device)
+    gpu_index = int(os.environ.get("CUDA_VISIBLE_DEVICES", str(local)).split(",")[local]) \
+        if os.environ.get("CUDA_VISIBLE_DEVICES") else local
+
+    wl = build_workload(args.workload)
+    r = measure_ours(wl, args.steps, args.warmup, device, gpu_index)
+    work = step_work(wl, r["step_tokens"], r["step_pairs"])
+    ms_step = reduce_max(r["ms_total"], device) / args.steps
+    tokens_all = reduce_sum(float(wl.num_q_tokens), device)
+    e2e_ms = reduce_max(r["e2e_ms"], device) / args.steps
+    attn_ms = statistics.mean(r["attn_ms"])
+    achieved = work["attn_bytes"] / (attn_ms * 1e-3) / 1e9
+    digest = _sources_digest()
+    traffic = NCU_TRAFFIC.get(wl.name) if NCU_TRAFFIC.get("sources") == digest else None
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        cpu, _ = time_oracle(wl, budget_s=12.0)
+
+    if world > 1:
+        import torch.distributed as dist
+        dist.destroy_process_group()
+    if rank != 0:
+        return 0
+    roof = {"kernel": "pa_attention (paged_decode_kernel + decode_combine_kernel%s)"
+                      % (" + paged_prefill_kernel" if wl.max_query_len > 1 else ""),
+            "bound": "hbm", "achieved": achieved, "peak": hbm_peak, "unit": "GB/s",
+            "frac": achieved / hbm_peak, "traffic": traffic, "peak_source": peak_src + " (MEASURED_PEAKS.json hbm_gbs)"
+            if peak_src == "measured" else "fallback 6.65 TB/s",
+            "algorithmic_bytes_per_launch": work["attn_bytes"], "launch_ms": attn_ms,
+            "kv_read_gbs": work["attn_kv_bytes"] / (attn_ms * 1e-3) / 1e9}
+    if work["prefill_flops"]:
+        roof["prefill_flops_per_launch"] = work["prefill_flops"]
+        roof["tensor_frac_of_bf16_peak"] = work["prefill_flops"] / (attn_ms * 1e-3) / 1e12 / bf16_peak
+    line = {"metric": METRIC, "value": tokens_all / (ms_step * 1e-3), "unit": UNIT, "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "bf16" if wl.geometry.dtype == "bf16" else "fp32",
+            "data": "synthetic (seeded N(0,1) K/V/Q, random-init; no dataset)",
+            "config": workload_config(wl, world, "KV read per step %.0f MB > 126 MB L2; no flush"
+                                      % (work["attn_kv_bytes"] / 1e6)),
+            "roofline": roof, "cpu_baseline": cpu,
+            "e2e": {"value": tokens_all / (e2e_ms * 1e-3), "unit": UNIT, "h2d_bytes_per_step": r["h2d"],
+                    "d2h_bytes_per_step": r["d2h"], "ms_per_step": e2e_ms},
+            "gpu_launches": r["launches"], "clocks": r["clocks"], "device_flags": r["flags"],
+            "step_bytes": work["attn_bytes"] + work["store_bytes"] + work["copy_bytes"]}
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+if __name__ == "__main__":
+    sys.exit(main())

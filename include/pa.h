@@ -1,0 +1,224 @@
+/*
+ * pa.h -- C ABI of libpa, the paged KV-cache hot path for NVIDIA B200 (sm_100a).
+ *
+ * Pages this interface restates (titles as published):
+ *   [A] "深入剖析nano-vLLM推理引擎架构：PagedAttention内存管理实现"
+ *   [B] "深入解析 nano-vLLM 推理引擎的分页 KV 缓存与内存优化架构"
+ *   [C] "vLLM核心架构：PagedAttention原理、KV Cache管理、连续批处理机制"
+ *
+ * Cache layout (all calls): K and V caches are separate, contiguous arrays
+ *   [num_blocks, block_size, num_kv_heads, head_dim]
+ * of the cache dtype. Slot s is row s of the flat view
+ *   [num_blocks * block_size, num_kv_heads * head_dim]
+ * ([B] §"分页 KV 缓存的核心机制" flattens the cache to slots; the heads axis is kept).
+ *
+ * Conventions shared by every call:
+ *  - Ownership: the caller owns every buffer, host and device. The library
+ *    never allocates device memory; the only library-owned object is the
+ *    host-side block manager handle (pa_bm_create / pa_bm_destroy).
+ *  - Streams: `stream` is a cudaStream_t passed as void* (NULL = legacy
+ *    default stream). Kernel calls are asynchronous and never synchronise the
+ *    host, except pa_read_device_flags, which says so.
+ *  - Errors: arguments are checked on the host before anything is launched; a
+ *    failed check returns a non-zero pa_status and launches nothing.
+ *    pa_last_error() gives a message for the calling thread's last failure.
+ *  - Device-side index checks: index *contents* (slots, block ids, context
+ *    lengths, copy pairs) live in device memory and cannot be checked before
+ *    launch. Kernels range-check each index they use; an out-of-range index
+ *    is skipped (no memory access) and a bit is set in the library's device
+ *    status word (PA_FLAG_*), read with pa_read_device_flags. No kernel traps.
+ *  - All indices are int32. Block-table rows are padded with -1; a negative
+ *    slot means a padding token.
+ */
+#ifndef PA_H_
+#define PA_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  PA_OK = 0,
+  PA_ERR_INVALID_ARG = 1,   /* null pointer, negative count, inconsistent sizes */
+  PA_ERR_UNSUPPORTED = 2,   /* valid but not implemented (dtype, head_dim, block_size...) */
+  PA_ERR_CUDA = 3,          /* a CUDA runtime / driver call failed; see pa_last_error */
+  PA_ERR_OUT_OF_BLOCKS = 4, /* block manager: free list too short; state unchanged */
+  PA_ERR_INDEX = 5          /* block manager: unknown sequence or bad position */
+} pa_status;
+
+typedef enum { PA_FP32 = 0, PA_BF16 = 1 } pa_dtype;
+
+/* Geometry of one K or V cache (both caches share it). Supported:
+ * dtype PA_BF16 or PA_FP32; head_dim 64 or 128; block_size 8, 16 or 32;
+ * num_kv_heads >= 1; num_blocks >= 1. */
+typedef struct {
+  int32_t num_blocks;
+  int32_t block_size;
+  int32_t num_kv_heads;
+  int32_t head_dim;
+  int32_t dtype; /* pa_dtype */
+} pa_cache_desc;
+
+/* Bits of the device status word (pa_read_device_flags). */
+#define PA_FLAG_SLOT_RANGE 0x1u    /* pa_store_kv: slot >= num_blocks * block_size */
+#define PA_FLAG_BLOCK_RANGE 0x2u   /* pa_attention: block id outside [0, num_blocks) */
+#define PA_FLAG_CONTEXT_RANGE 0x4u /* pa_attention: context_len > max_context_len or
+                                      max_blocks_per_seq * block_size, or q_len > context_len */
+#define PA_FLAG_PAIR_RANGE 0x8u    /* pa_copy_blocks: src or dst outside [0, num_blocks) */
+#define PA_FLAG_WAIT_TIMEOUT 0x10u /* a bounded device-side wait gave up */
+
+/* ------------------------------------------------------------------ kernels */
+
+/*
+ * pa_store_kv -- slot-mapped KV write ([B] §"分页 KV 缓存的核心机制"; blocks are
+ * filled as tokens arrive, [A] §"PagedAttention：操作系统的内存智慧").
+ *   k, v          device, [num_tokens, num_kv_heads, head_dim], cache dtype, contiguous
+ *   slot_mapping  device int32 [num_tokens]; token t goes to slot slot_mapping[t];
+ *                 negative = skip. Two tokens of one call must not share a slot.
+ *   k_cache, v_cache  device caches (layout above), written in place.
+ * A bit copy: cache rows receive exactly the bits of k and v.
+ * Slots >= num_blocks*block_size are skipped and raise PA_FLAG_SLOT_RANGE.
+ * num_tokens == 0 is a no-op.
+ */
+pa_status pa_store_kv(const void* k, const void* v, const int32_t* slot_mapping, int32_t num_tokens,
+                      void* k_cache, void* v_cache, const pa_cache_desc* cache, void* stream);
+
+/*
+ * pa_copy_blocks -- copy-on-write block copy ([C] §"二、KV Cache管理：从浪费到极致复用":
+ * a shared page is copied only when a request writes it, as in fork).
+ *   src_dst_pairs device int32 [num_pairs, 2]; for each pair, block dst of
+ *                 both caches becomes a copy of block src.
+ * No dst may repeat or also appear as a src within one call (the block manager
+ * never produces that); pairs with src == dst are no-ops. Out-of-range ids are
+ * skipped and raise PA_FLAG_PAIR_RANGE. num_pairs == 0 is a no-op.
+ */
+pa_status pa_copy_blocks(const int32_t* src_dst_pairs, int32_t num_pairs, void* k_cache,
+                         void* v_cache, const pa_cache_desc* cache, void* stream);
+
+/*
+ * pa_attention_workspace_size -- bytes of device workspace pa_attention needs
+ * for these sizes (0 when no sequence can be split). Same arguments as the
+ * matching pa_attention call. Returns 0 for invalid arguments too; the
+ * matching pa_attention call then reports the error.
+ */
+size_t pa_attention_workspace_size(int32_t num_seqs, int32_t num_q_heads, int32_t max_query_len,
+                                   int32_t max_context_len, const pa_cache_desc* cache);
+
+/*
+ * pa_attention -- attention of every query row over its sequence's keys,
+ * gathered through the block table ([A] §"PagedAttention：操作系统的内存智慧",
+ * [C] §"一、PagedAttention：虚拟内存的灵感"; prefill rows and decode rows,
+ * [B] §"工程落地：配置参数与监控指标").
+ *   q                device [num_q_tokens, num_q_heads, head_dim], cache dtype
+ *   k_cache, v_cache device caches (read only)
+ *   block_tables     device int32 [num_seqs, max_blocks_per_seq], row s maps
+ *                    logical block i of sequence s to a physical block
+ *   context_lens     device int32 [num_seqs]; L_s counts every key of
+ *                    sequence s, including the rows queried now (store first)
+ *   query_start_loc  device int32 [num_seqs + 1]; sequence s owns query rows
+ *                    query_start_loc[s] .. query_start_loc[s+1]-1
+ *   max_query_len    host bound on q_len_s (1 => decode-only batch)
+ *   max_context_len  host bound on L_s; rows of a sequence with a larger L_s
+ *                    are left unwritten and raise PA_FLAG_CONTEXT_RANGE
+ *   scale            softmax scale (usually 1/sqrt(head_dim))
+ *   out              device [num_q_tokens, num_q_heads, head_dim], cache dtype
+ *   workspace        device scratch of at least pa_attention_workspace_size()
+ *                    bytes (may be NULL when that is 0); contents are
+ *                    overwritten; not shared by concurrent calls.
+ * Row j of sequence s sits at position p = L_s - q_len_s + j and attends keys
+ * 0..p; query head h uses KV head h / (num_q_heads / num_kv_heads).
+ * num_q_heads must be a multiple of num_kv_heads. Rows with q_len_s > 1 need a
+ * bf16 cache (tcgen05 tensor-core path); fp32 supports decode rows only.
+ * Sequences with q_len_s == 0 are skipped. Rows of `out` not owned by any
+ * sequence are not written.
+ */
+pa_status pa_attention(const void* q, const void* k_cache, const void* v_cache,
+                       const int32_t* block_tables, int32_t max_blocks_per_seq,
+                       const int32_t* context_lens, const int32_t* query_start_loc,
+                       int32_t num_seqs, int32_t num_q_tokens, int32_t num_q_heads,
+                       int32_t max_query_len, int32_t max_context_len, float scale,
+                       const pa_cache_desc* cache, void* out, void* workspace,
+                       size_t workspace_bytes, void* stream);
+
+/*
+ * pa_read_device_flags -- read (and optionally clear) the device status word
+ * of the current device. Synchronises the device first (all streams).
+ *   flags  host out: OR of PA_FLAG_* raised since the last clear
+ *   clear  non-zero: reset the word to 0 after reading
+ */
+pa_status pa_read_device_flags(uint32_t* flags, int32_t clear);
+
+/* Message for the calling thread's last non-OK status ("" if none). */
+const char* pa_last_error(void);
+
+/* Library version string. */
+const char* pa_version(void);
+
+/* ------------------------------------------------------------ block manager */
+
+/*
+ * Host-side block manager: free list, per-sequence block tables, reference
+ * counts and copy-on-write ([A] §"PagedAttention：操作系统的内存智慧": free list
+ * and block table, a new block only when the current one is full; [A]
+ * §"连续批处理与内存管理的协同": a finished request returns its blocks; [C]
+ * §"二、KV Cache管理：从浪费到极致复用": shared prefix pages, reference counts,
+ * copy-on-write). It only produces int32 index arrays in host memory; it never
+ * touches the GPU. Allocation takes blocks from the front of the free list,
+ * freed blocks go to its back. A failing call changes no state.
+ * A handle is not thread-safe; distinct handles are independent.
+ */
+typedef struct pa_bm pa_bm;
+
+/* initial_free_order: host int32 [num_blocks], a permutation of 0..num_blocks-1
+ * giving the initial free-list order, or NULL for 0, 1, 2, ... */
+pa_status pa_bm_create(int32_t num_blocks, int32_t block_size, const int32_t* initial_free_order,
+                       pa_bm** out);
+void pa_bm_destroy(pa_bm* bm);
+
+/* New sequence holding num_tokens tokens (ceil(num_tokens/block_size) blocks).
+ * slots_out: host int32 [num_tokens] receiving the slot of each token, or NULL. */
+pa_status pa_bm_add_seq(pa_bm* bm, int64_t seq_id, int32_t num_tokens, int32_t* slots_out);
+
+/* child shares the blocks holding parent's first num_tokens tokens (refcount +1
+ * each); num_tokens < 0 means all of parent's tokens. */
+pa_status pa_bm_fork(pa_bm* bm, int64_t parent, int64_t child, int32_t num_tokens);
+
+/* Append n tokens. slots_out: host int32 [n] (or NULL). If the last block is
+ * partly filled and shared, it is replaced by a fresh block and the pair
+ * (old, new) is written to cow_pair_out (host int32 [2], may be NULL) with
+ * *num_cow_out = 1 (else 0); the caller copies old -> new (pa_copy_blocks)
+ * before storing the new rows. */
+pa_status pa_bm_append_tokens(pa_bm* bm, int64_t seq_id, int32_t n, int32_t* slots_out,
+                              int32_t* cow_pair_out, int32_t* num_cow_out);
+
+/* Drop the sequence; each of its blocks loses one reference and goes back to
+ * the free list when it reaches 0 (in logical order). */
+pa_status pa_bm_free_seq(pa_bm* bm, int64_t seq_id);
+
+/* Slots of positions [start, start+n) of a sequence. out: host int32 [n]. */
+pa_status pa_bm_slot_mapping(const pa_bm* bm, int64_t seq_id, int32_t start, int32_t n,
+                             int32_t* out);
+
+/* Block table rows for n sequences: table_out host int32 [n, max_blocks]
+ * padded with -1; ctx_lens_out host int32 [n] (may be NULL). Fails with
+ * PA_ERR_INVALID_ARG if a sequence holds more than max_blocks blocks. */
+pa_status pa_bm_block_table(const pa_bm* bm, const int64_t* seq_ids, int32_t n, int32_t max_blocks,
+                            int32_t* table_out, int32_t* ctx_lens_out);
+
+int32_t pa_bm_num_free(const pa_bm* bm);
+int32_t pa_bm_num_blocks(const pa_bm* bm);
+/* Reference count of a block, or -1 if out of range. */
+int32_t pa_bm_refcount(const pa_bm* bm, int32_t block);
+/* Tokens held by a sequence, or -1 if unknown. */
+int32_t pa_bm_seq_len(const pa_bm* bm, int64_t seq_id);
+/* Copy up to cap free-list entries (front first) to out; returns the count. */
+int32_t pa_bm_free_list(const pa_bm* bm, int32_t* out, int32_t cap);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* PA_H_ */

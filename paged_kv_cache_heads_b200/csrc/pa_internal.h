@@ -1,0 +1,79 @@
+// Internal launcher interface between the C-ABI layer (pa_api.cu) and the
+// kernel translation units. Host code only; no torch types anywhere.
+#pragma once
+
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <stddef.h>
+#include <stdint.h>
+
+#include "pa.h"
+
+namespace pa {
+
+// Device-side work description of one pa_attention call (decode part).
+struct DecodeArgs {
+  const void* q;
+  void* out;
+  const int32_t* block_tables;
+  const int32_t* context_lens;
+  const int32_t* query_start_loc;
+  float* part_o;     // [num_seqs][max_splits][num_q_heads][head_dim] fp32 (or null)
+  float* part_lse;   // [num_seqs][max_splits][num_q_heads] fp32, log2 domain (or null)
+  unsigned* status;  // library status word
+  int32_t max_blocks_per_seq;
+  int32_t num_seqs;
+  int32_t num_q_heads;
+  int32_t num_kv_heads;
+  int32_t num_blocks;
+  int32_t max_context_len;
+  int32_t chunk_tokens;  // upper bound on keys per split (multiple of block_size)
+  int32_t max_splits;    // ceil(max_context_len / chunk_tokens)
+  float scale_log2;      // scale * log2(e)
+};
+
+struct PrefillArgs {
+  void* out;
+  const int32_t* block_tables;
+  const int32_t* context_lens;
+  const int32_t* query_start_loc;
+  unsigned* status;
+  int32_t max_blocks_per_seq;
+  int32_t num_seqs;
+  int32_t num_q_heads;
+  int32_t num_kv_heads;
+  int32_t num_blocks;
+  int32_t max_context_len;
+  int32_t max_query_len;
+  int32_t num_q_tokens;
+  float scale_log2;
+};
+
+// Sets the calling thread's pa_last_error() message.
+void set_last_error(const char* msg);
+
+// Split policy shared by the workspace size query and the launch.
+int32_t decode_chunk_tokens(int32_t num_seqs, int32_t num_kv_heads, int32_t group,
+                            int32_t max_context_len, int32_t block_size);
+inline int32_t ceil_div(int64_t a, int64_t b) { return static_cast<int32_t>((a + b - 1) / b); }
+
+// Launchers return cudaSuccess or the launch error. `maps` are encoded tensor
+// maps for the K and V caches (box and swizzle as the kernel requires).
+cudaError_t launch_store_kv(const void* k, const void* v, const int32_t* slots, int32_t num_tokens,
+                            void* k_cache, void* v_cache, const pa_cache_desc& c, unsigned* status,
+                            cudaStream_t stream);
+cudaError_t launch_copy_blocks(const int32_t* pairs, int32_t num_pairs, void* k_cache,
+                               void* v_cache, const pa_cache_desc& c, unsigned* status,
+                               cudaStream_t stream);
+cudaError_t launch_decode(const DecodeArgs& a, const CUtensorMap& kmap, const CUtensorMap& vmap,
+                          const pa_cache_desc& c, cudaStream_t stream);
+cudaError_t launch_decode_combine(const DecodeArgs& a, const pa_cache_desc& c, cudaStream_t stream);
+cudaError_t launch_prefill(const PrefillArgs& a, const CUtensorMap& qmap, const CUtensorMap& kmap,
+                           const CUtensorMap& vmap, const pa_cache_desc& c, cudaStream_t stream);
+
+// Heads of one GQA group handled together by one decode CTA.
+int32_t decode_heads_per_cta(int32_t group);
+// Decode smem stage geometry, used by the launcher and the API's checks.
+int32_t num_sms();
+
+}  // namespace pa

@@ -1,0 +1,229 @@
+"""C-ABI checks that need no GPU: exports, host-side validation, block manager parity.
+
+The block manager in libpa (C++) is compared bit-exactly with the oracle's
+(Python) on the workloads and on random operation sequences: slots, copy
+pairs, block tables, free-list order and reference counts.
+"""
+
+import os
+import re
+import subprocess
+import sys
+
+import numpy as np
+import pytest
+
+import oracle
+import paged_kv_cache_heads_b200 as P
+from paged_kv_cache_heads_b200 import workloads as W
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+pytestmark = pytest.mark.skipif(not os.path.exists(P.library_path()), reason="libpa.so not built")
+
+
+def header_functions():
+    text = open(os.path.join(ROOT, "include", "pa.h")).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(pa_\w+)\s*\(", text)))
+
+
+def test_library_exports_every_declared_entry_point():
+    import ctypes
+    lib = ctypes.CDLL(P.library_path())
+    declared = header_functions()
+    assert len(declared) >= 20
+    for name in declared:
+        assert hasattr(lib, name), name
+    assert sorted(P.exported_symbols()) == declared
+
+
+def test_missing_library_fails_loudly():
+    code = ("import paged_kv_cache_heads_b200 as P\n"
+            "try:\n    P.pa_version()\nexcept RuntimeError as e:\n    print('LOUD', e)\n")
+    env = dict(os.environ, PA_LIBRARY="/nonexistent/libpa.so")
+    r = subprocess.run([sys.executable, "-c", code], capture_output=True, text=True, env=env, cwd=ROOT)
+    assert "LOUD" in r.stdout and "libpa.so not found" in r.stdout
+
+
+FAKE = 0x10000  # aligned non-null address; validation must reject before any use
+DESC = (64, 16, 8, 128, P.PA_BF16)
+
+
+@pytest.mark.parametrize("desc,status", [
+    ((64, 16, 8, 96, P.PA_BF16), P.PA_ERR_UNSUPPORTED),     # head_dim
+    ((64, 64, 8, 128, P.PA_BF16), P.PA_ERR_UNSUPPORTED),    # block_size
+    ((64, 16, 8, 128, 7), P.PA_ERR_UNSUPPORTED),            # dtype
+    ((0, 16, 8, 128, P.PA_BF16), P.PA_ERR_INVALID_ARG),     # empty pool
+    ((64, 16, 0, 128, P.PA_BF16), P.PA_ERR_INVALID_ARG),    # no heads
+])
+def test_bad_cache_descriptor_rejected(desc, status):
+    with pytest.raises(P.PAError) as e:
+        P.pa_store_kv(FAKE, FAKE, FAKE, 4, FAKE, FAKE, desc, stream=0)
+    assert e.value.status == status
+
+
+def test_store_and_copy_validation():
+    with pytest.raises(P.PAError) as e:
+        P.pa_store_kv(None, FAKE, FAKE, 4, FAKE, FAKE, DESC, stream=0)
+    assert e.value.status == P.PA_ERR_INVALID_ARG
+    with pytest.raises(P.PAError) as e:
+        P.pa_store_kv(FAKE + 8, FAKE, FAKE, 4, FAKE, FAKE, DESC, stream=0)   # misaligned
+    assert e.value.status == P.PA_ERR_INVALID_ARG
+    with pytest.raises(P.PAError):
+        P.pa_store_kv(FAKE, FAKE, FAKE, -1, FAKE, FAKE, DESC, stream=0)
+    P.pa_store_kv(None, None, None, 0, None, None, DESC, stream=0)          # empty call is a no-op
+    P.pa_copy_blocks(None, 0, None, None, DESC, stream=0)
+    with pytest.raises(P.PAError):
+        P.pa_copy_blocks(None, 3, FAKE, FAKE, DESC, stream=0)
+
+
+def _attn(**kw):
+    args = dict(q=FAKE, k_cache=FAKE, v_cache=FAKE, block_tables=FAKE, max_blocks_per_seq=128,
+                context_lens=FAKE, query_start_loc=FAKE, num_seqs=4, num_q_tokens=4, num_q_heads=32,
+                max_query_len=1, max_context_len=2048, scale=0.088, cache=DESC, out=FAKE,
+                workspace=None, workspace_bytes=0, stream=0)
+    args.update(kw)
+    return P.pa_attention(**args)
+
+
+def test_attention_validation():
+    with pytest.raises(P.PAError) as e:
+        _attn(num_q_heads=30)                                  # not a multiple of 8 kv heads
+    assert e.value.status == P.PA_ERR_INVALID_ARG
+    with pytest.raises(P.PAError) as e:
+        _attn()                                                # splits need a workspace
+    assert e.value.status == P.PA_ERR_INVALID_ARG and "workspace" in str(e.value)
+    need = P.pa_attention_workspace_size(4, 32, 1, 2048, DESC)
+    with pytest.raises(P.PAError):
+        _attn(workspace=FAKE, workspace_bytes=need - 1)
+    with pytest.raises(P.PAError) as e:
+        _attn(max_query_len=2, cache=(64, 16, 8, 128, P.PA_FP32))
+    assert e.value.status == P.PA_ERR_UNSUPPORTED
+    with pytest.raises(P.PAError):
+        _attn(out=None)
+    with pytest.raises(P.PAError):
+        _attn(max_query_len=5)                                 # more than num_q_tokens
+    _attn(num_seqs=0)                                          # empty batch: no-op
+    _attn(num_q_tokens=0)
+
+
+def test_workspace_size_policy():
+    small = P.pa_attention_workspace_size(4, 32, 1, 32, DESC)
+    assert small == 0                                          # one split per sequence
+    big = P.pa_attention_workspace_size(32, 32, 1, 2048, (8192, 16, 32, 128, P.PA_BF16))
+    assert big > 0 and big % 4 == 0
+    assert P.pa_attention_workspace_size(4, 30, 1, 2048, DESC) == 0   # invalid -> 0
+    assert P.pa_attention_workspace_size(4, 32, 0, 2048, DESC) == 0   # nothing to do
+
+
+# --------------------------------------------------------------------------
+# libpa block manager == oracle block manager
+# --------------------------------------------------------------------------
+
+def _same_state(a: P.BlockManager, b: oracle.BlockManager, live):
+    assert a.free_list() == list(b.free)
+    assert [a.refcount(i) for i in range(b.num_blocks)] == list(b.ref)
+    for s in live:
+        assert a.seq_len(s) == b.seq_len(s)
+    if live:
+        mb = max(len(b.blocks_of(s)) for s in live) + 1
+        ta, la = a.block_table(live, mb)
+        tb, lb = b.block_table(live, mb)
+        assert np.array_equal(ta, tb) and np.array_equal(la, lb)
+
+
+@pytest.mark.parametrize("seed", range(8))
+def test_block_manager_matches_oracle_on_random_ops(seed):
+    rng = np.random.default_rng(500 + seed)
+    bs = int(rng.choice([8, 16, 32]))
+    nb = int(rng.integers(4, 96))
+    order = rng.permutation(nb)
+    a, b = P.BlockManager(nb, bs, order), oracle.BlockManager(nb, bs, order)
+    live, nid = [], 0
+    for _ in range(400):
+        r = rng.random()
+        if r < 0.25 or not live:
+            n = int(rng.integers(0, 3 * bs))
+            ra = rb = None
+            try:
+                rb = b.add_seq(nid, n)
+            except oracle.OutOfBlocks:
+                rb = "oob"
+            try:
+                ra = a.add_seq(nid, n)
+            except P.PAError as e:
+                assert e.status == P.PA_ERR_OUT_OF_BLOCKS
+                ra = "oob"
+            assert ra == rb
+            if rb != "oob":
+                live.append(nid)
+            nid += 1
+        elif r < 0.4:
+            par = int(rng.choice(live))
+            n = int(rng.integers(0, b.seq_len(par) + 1))
+            a.fork(par, nid, n)
+            b.fork(par, nid, n)
+            live.append(nid)
+            nid += 1
+        elif r < 0.85:
+            s = int(rng.choice(live))
+            n = int(rng.integers(0, 2 * bs + 3))
+            try:
+                rb = b.append_tokens(s, n)
+            except oracle.OutOfBlocks:
+                rb = "oob"
+            try:
+                ra = a.append_tokens(s, n)
+            except P.PAError as e:
+                assert e.status == P.PA_ERR_OUT_OF_BLOCKS
+                ra = "oob"
+            if rb == "oob":
+                assert ra == "oob"
+            else:
+                assert ra[0] == rb[0] and [tuple(p) for p in ra[1]] == [tuple(p) for p in rb[1]]
+        else:
+            s = int(rng.choice(live))
+            a.free_seq(s)
+            b.free_seq(s)
+            live.remove(s)
+        _same_state(a, b, live)
+    for s in live:
+        assert a.slot_mapping(s, 0, b.seq_len(s)) == b.slot_mapping(s, 0, b.seq_len(s))
+
+
+@pytest.mark.parametrize("name", ["tiny", "prefix_cow", "mixed_bs8"])
+def test_block_manager_matches_oracle_on_workloads(name):
+    wl = W.CONFIGS[name]()
+    geo = wl.geometry
+    a = P.BlockManager(geo.num_blocks, geo.block_size, wl.initial_free_order)
+    b = oracle.BlockManager(geo.num_blocks, geo.block_size, wl.initial_free_order)
+    for op in wl.ops:
+        if op.kind == "add":
+            assert a.add_seq(op.seq, op.n) == b.add_seq(op.seq, op.n)
+        elif op.kind == "fork":
+            a.fork(op.parent, op.seq, op.n)
+            b.fork(op.parent, op.seq, op.n)
+        elif op.kind == "append":
+            sa, pa_ = a.append_tokens(op.seq, op.n)
+            sb, pb = b.append_tokens(op.seq, op.n)
+            assert sa == sb and [tuple(p) for p in pa_] == [tuple(p) for p in pb]
+    _same_state(a, b, wl.batch_seqs)
+
+
+def test_block_manager_errors():
+    bm = P.BlockManager(4, 16)
+    with pytest.raises(P.PAError) as e:
+        bm.free_seq(3)
+    assert e.value.status == P.PA_ERR_INDEX
+    bm.add_seq(1, 20)
+    with pytest.raises(P.PAError):
+        bm.add_seq(1, 1)                                       # duplicate id
+    with pytest.raises(P.PAError) as e:
+        bm.append_tokens(1, 60)                                # needs 4 more, 2 free
+    assert e.value.status == P.PA_ERR_OUT_OF_BLOCKS and bm.seq_len(1) == 20 and bm.num_free() == 2
+    with pytest.raises(P.PAError):
+        bm.block_table([1], 1)                                 # holds 2 blocks
+    with pytest.raises(P.PAError):
+        P.BlockManager(3, 16, [0, 0, 1])                       # not a permutation
+    assert bm.refcount(99) == -1 and bm.seq_len(42) == -1

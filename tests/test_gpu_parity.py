@@ -1,0 +1,161 @@
+"""GPU parity: libpa against the oracle on the same seeded workloads.
+
+Store, copy and all block-table / slot indexing must match bit for bit;
+attention must be within max |err| 2e-2 and mean |err| 2e-3 of the fp64
+oracle for bf16 inputs (fp32 accumulation), and within 1e-4 for fp32 inputs.
+The named configurations run at full size through the same calls the bench
+times; the random sweep covers every supported dtype / head_dim / block size
+and GQA grouping with ragged lengths and multi-split sequences.
+"""
+
+import os
+
+import numpy as np
+import pytest
+
+import oracle
+from oracle import scenario as oscen
+from paged_kv_cache_heads_b200 import workloads as W
+
+pytestmark = pytest.mark.gpu
+
+TOL = {W.BF16: (2e-2, 2e-3), W.FP32: (1e-4, 1e-5)}
+
+
+@pytest.fixture(scope="module")
+def P():
+    import torch
+    if not torch.cuda.is_available():
+        pytest.skip("no CUDA device")
+    import paged_kv_cache_heads_b200 as P
+    P.load_library()
+    P.pa_read_device_flags(clear=True)
+    return P
+
+
+def _check_attention(got, ref, dtype, ctx=""):
+    amax, amean = TOL[dtype]
+    err = np.abs(got - ref)
+    assert np.isfinite(got).all(), "non-finite output " + ctx
+    assert err.max() <= amax, "max err %.3g %s" % (err.max(), ctx)
+    assert err.mean() <= amean, "mean err %.3g %s" % (err.mean(), ctx)
+    return float(err.max()), float(err.mean())
+
+
+def _run_both(P, wl, check_caches=True):
+    import torch
+    from paged_kv_cache_heads_b200 import scenario as gs
+    b = gs.prepare(wl)
+    gs.run_step(b)
+    torch.cuda.synchronize()
+    kc, vc = W.sentinel_cache(wl.geometry), W.sentinel_cache(wl.geometry)
+    o = oscen.run(wl, kc, vc)
+    # indexing: identical slots, copy pairs, tables and lengths
+    assert b.host["op_slots"] == [list(map(int, s)) for s in o.op_slots]
+    assert [[tuple(p) for p in ps] for ps in b.host["op_pairs"]] == [[tuple(p) for p in ps] for ps in o.op_pairs]
+    assert np.array_equal(b.host["block_tables"], o.block_tables)
+    assert np.array_equal(b.host["context_lens"], o.context_lens)
+    if check_caches:
+        want_k = o.k_cache.view(np.uint16 if wl.geometry.dtype == W.BF16 else np.uint32)
+        want_v = o.v_cache.view(np.uint16 if wl.geometry.dtype == W.BF16 else np.uint32)
+        assert np.array_equal(gs.cache_bits(b.k_cache), want_k)
+        assert np.array_equal(gs.cache_bits(b.v_cache), want_v)
+    got = gs.out_as_f64(b.out, wl.geometry.dtype)
+    flags = P.pa_read_device_flags(clear=True)
+    assert flags == 0, hex(flags)
+    return b, o, got
+
+
+@pytest.mark.parametrize("name", ["tiny", "llama7b", "gqa_long", "prefix_cow", "prefix_cow_p2000"])
+def test_config_parity(P, name):
+    wl = W.prefix_cow_decode(prefix_len=2000) if name == "prefix_cow_p2000" else W.CONFIGS[name]()
+    b, o, got = _run_both(P, wl)
+    _check_attention(got, o.out, wl.geometry.dtype, name)
+    if name == "prefix_cow":
+        assert sum(len(p) for p in o.op_pairs) == 47
+    if name == "prefix_cow_p2000":
+        assert sum(len(p) for p in o.op_pairs) == 0
+
+
+def _random_decode(seed, dtype, d, bs, g, hkv=2, nseq=7):
+    rng = np.random.default_rng(seed)
+    lens = [1, bs, bs + 1, int(rng.integers(2, 3 * bs)), int(rng.integers(600, 1400)),
+            int(rng.integers(1, 64)), int(rng.integers(2000, 2600))][:nseq]
+    return W.random_case(seed, num_seqs=len(lens), q_lens=[1] * len(lens), ctx_extra=[x - 1 for x in lens],
+                         num_kv_heads=hkv, group=g, head_dim=d, block_size=bs, dtype=dtype)
+
+
+@pytest.mark.parametrize("dtype", [W.BF16, W.FP32])
+@pytest.mark.parametrize("d", [64, 128])
+@pytest.mark.parametrize("bs", [8, 16, 32])
+@pytest.mark.parametrize("g", [1, 2, 3, 4, 8])
+def test_random_decode_sweep(P, dtype, d, bs, g):
+    wl = _random_decode(1000 + d + bs + 7 * g, dtype, d, bs, g)
+    b, o, got = _run_both(P, wl)
+    _check_attention(got, o.out, dtype, "dtype=%s d=%d bs=%d g=%d" % (dtype, d, bs, g))
+
+
+@pytest.mark.parametrize("chunk", ["16", "64", "512"])
+def test_split_count_does_not_change_result(P, chunk, monkeypatch):
+    monkeypatch.setenv("PA_DECODE_CHUNK", chunk)
+    wl = _random_decode(77, W.BF16, 128, 16, 4)
+    b, o, got = _run_both(P, wl, check_caches=False)
+    _check_attention(got, o.out, W.BF16, "chunk " + chunk)
+
+
+def test_empty_and_zero_length_query_rows(P):
+    import torch
+    from paged_kv_cache_heads_b200 import scenario as gs
+    wl = W.random_case(5, num_seqs=4, q_lens=[1, 0, 1, 0], ctx_extra=[9, 30, 0, 3], num_kv_heads=2,
+                       group=2, head_dim=64, block_size=16, dtype=W.BF16)
+    b = gs.prepare(wl)
+    gs.run_step(b)
+    torch.cuda.synchronize()
+    o = oscen.run(wl, W.sentinel_cache(wl.geometry), W.sentinel_cache(wl.geometry))
+    _check_attention(gs.out_as_f64(b.out, W.BF16), o.out, W.BF16)
+    assert P.pa_read_device_flags(clear=True) == 0
+
+
+def test_out_of_range_indices_are_flagged_not_followed(P):
+    import torch
+    from paged_kv_cache_heads_b200 import scenario as gs
+    dev = "cuda"
+    geo = W.Geometry(8, 16, 2, 4, 64, W.BF16, 4)
+    desc = gs.cache_desc(geo)
+    kc = gs.sentinel_cache_dev(geo, dev)
+    vc = gs.sentinel_cache_dev(geo, dev)
+    k = torch.ones((3, 2, 64), dtype=torch.int16, device=dev)
+    slots = torch.tensor([5, 8 * 16, -1], dtype=torch.int32, device=dev)   # middle one is out of range
+    P.pa_store_kv(k, k, slots, 3, kc, vc, desc)
+    assert P.pa_read_device_flags(clear=True) == P.PA_FLAG_SLOT_RANGE
+    bits = gs.cache_bits(kc).reshape(8 * 16, -1)
+    assert (bits[5] == 1).all()
+    assert (np.delete(bits, 5, axis=0) == W.SENTINEL_BF16).all()
+    pairs = torch.tensor([[0, 1], [2, 99]], dtype=torch.int32, device=dev)
+    P.pa_copy_blocks(pairs, 2, kc, vc, desc)
+    assert P.pa_read_device_flags(clear=True) == P.PA_FLAG_PAIR_RANGE
+    q = torch.zeros((2, 4, 64), dtype=torch.int16, device=dev)
+    out = torch.zeros_like(q)
+    tables = torch.tensor([[0, 77, -1, -1], [1, 2, 3, -1]], dtype=torch.int32, device=dev)
+    lens = torch.tensor([20, 70], dtype=torch.int32, device=dev)       # seq 1 exceeds max_context_len
+    qsl = torch.tensor([0, 1, 2], dtype=torch.int32, device=dev)
+    P.pa_attention(q, kc, vc, tables, 4, lens, qsl, 2, 2, 4, 1, 48, 0.125, desc, out, None, stream=None)
+    flags = P.pa_read_device_flags(clear=True)
+    assert flags & P.PA_FLAG_BLOCK_RANGE and flags & P.PA_FLAG_CONTEXT_RANGE
+    assert not flags & P.PA_FLAG_WAIT_TIMEOUT
+    assert (out[1] == 0).all()                                         # rows of a rejected sequence untouched
+
+
+def test_repeated_step_is_idempotent(P):
+    import torch
+    from paged_kv_cache_heads_b200 import scenario as gs
+    wl = W.gqa_long_decode()
+    b = gs.prepare(wl)
+    gs.run_step(b)
+    first = b.out.clone()
+    k0 = gs.cache_bits(b.k_cache)
+    for _ in range(3):
+        gs.run_step(b)
+    torch.cuda.synchronize()
+    assert torch.equal(first, b.out)
+    assert np.array_equal(k0, gs.cache_bits(b.k_cache))
