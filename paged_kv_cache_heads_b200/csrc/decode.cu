@@ -88,8 +88,12 @@ struct DecodeCfg {
   static constexpr int kNIT = kSteps < 8 ? kSteps : 8;  // steps per softmax update
   static constexpr int kNUPD = kSteps / kNIT;
   static constexpr int kStageB = 2 * BS * kRowB;    // K block + V block
+  // Stages: about 64 KiB in flight, and a multiple of NCW so that every use of
+  // a stage belongs to the same consumer warp (its parity waits then never
+  // run more than one phase ahead of the barrier).
   static constexpr int kNST0 = 65536 / kStageB;
-  static constexpr int kNST = kNST0 < 2 ? 2 : (kNST0 > 16 ? 16 : kNST0);
+  static constexpr int kNST1 = kNST0 < NCW ? NCW : (kNST0 > 16 ? 16 : kNST0);
+  static constexpr int kNST = (kNST1 / NCW) * NCW;
   static constexpr int kThreads = (NCW + 1) * 32;
   static constexpr int kCombFloats = NCW * GH * (D + 2);
   // dynamic smem: stages | bars | comb x2 | warp totals | prefix, clen, row
@@ -100,6 +104,7 @@ struct DecodeCfg {
   static constexpr int kSeqOff = kAbortOff + 16;
   static_assert(kRowB % 16 == 0 && 32 % kLPR == 0, "row must split into lanes");
   static_assert(BS % kTPW == 0 && kSteps % kNIT == 0, "block must split into steps");
+  static_assert(kNST % NCW == 0, "each stage must always go to the same consumer warp");
   static size_t smem_bytes(int num_seqs) { return 1024 + kSeqOff + 12ull * (num_seqs + 1); }
 };
 

@@ -364,7 +364,7 @@ pa_status pa_attention(const void* q, const void* k_cache, const void* v_cache,
     const uint64_t qd[3] = {uint64_t(cache->head_dim), uint64_t(num_q_heads), uint64_t(num_q_tokens)};
     const uint64_t qs[2] = {uint64_t(cache->head_dim) * 2, uint64_t(num_q_heads) * cache->head_dim * 2};
     const int32_t g = num_q_heads / cache->num_kv_heads;
-    const int32_t gh = (g <= 16 && (g & (g - 1)) == 0) ? g : 1;
+    const int32_t gh = prefill_heads_per_tile(g);
     const uint32_t qbox[3] = {64, uint32_t(gh), uint32_t(128 / gh)};
     CUtensorMap qmap, pk, pv;
     if ((st = tensor_map(&qmap, q, 3, qd, qs, qbox, PA_BF16, 128)) != PA_OK) return st;

@@ -71,6 +71,8 @@ cudaError_t launch_decode_combine(const DecodeArgs& a, const pa_cache_desc& c, c
 cudaError_t launch_prefill(const PrefillArgs& a, const CUtensorMap& qmap, const CUtensorMap& kmap,
                            const CUtensorMap& vmap, const pa_cache_desc& c, cudaStream_t stream);
 
+// Query heads packed into one 128-row prefill tile (the rest of its rows are tokens).
+int32_t prefill_heads_per_tile(int32_t group);
 // Heads of one GQA group handled together by one decode CTA.
 int32_t decode_heads_per_cta(int32_t group);
 // Decode smem stage geometry, used by the launcher and the API's checks.

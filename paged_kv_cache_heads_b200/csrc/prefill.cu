@@ -1,12 +1,448 @@
-// Chunked-prefill attention (query rows of sequences with q_len > 1).
+// Chunked-prefill attention on the 5th-generation tensor cores (tcgen05).
+//
+// Rows of sequences with q_len > 1: row j of sequence s sits at position
+// p = L - q_len + j and attends keys 0..p (causal inside the chunk, full over
+// the cached context), keys gathered through the block table. This is the
+// prefill call that the page "深入解析 nano-vLLM 推理引擎的分页 KV 缓存与内存优化架构",
+// §"工程落地：配置参数与监控指标" hands to a variable-length attention kernel,
+// here on a paged cache with the 256-token prefill chunks of the page
+// "深入剖析nano-vLLM推理引擎架构：PagedAttention内存管理实现", §"可落地配置参数".
+//
+// Design (B200, one CTA per 128-row tile, persistent over tiles):
+//  * A tile holds 128 query rows: 128/GH tokens x the GH query heads of one
+//    GQA group, so each gathered K/V tile serves every head of the group.
+//  * Warp 4 (producer) loads the Q tile with one TMA per 64 head-dim columns
+//    and, per 64-key tile, each K/V block of the tile with TMA (box
+//    {64, 1, bs, 1}, 128-byte swizzle) into a 2-stage ring.
+//  * Thread 0 issues S = Q K^T (M=128, N=64, K=16 steps) into TMEM, then
+//    O += P V (M=128, N=head_dim) into TMEM; tcgen05.commit signals mbarriers.
+//  * Warps 0-3 own one row each (TMEM lane = row): load S, mask, online
+//    softmax in fp32 (exp2 with the scale folded into log2 e), write P as bf16
+//    into the K slot it no longer needs (128-byte swizzled K-major layout).
+//    O in TMEM is rescaled only when a row's running max grows by more than
+//    2^8, so most tiles skip the TMEM round trip.
+//  * V rows at or beyond L inside the last tile are zeroed before the PV MMA
+//    so stale bits in the unfilled tail of a block cannot reach the output.
+#include <math_constants.h>
+
 #include "pa_common.cuh"
 #include "pa_internal.h"
+#include "tcgen05.cuh"
 
 namespace pa {
+namespace {
 
-cudaError_t launch_prefill(const PrefillArgs&, const CUtensorMap&, const CUtensorMap&,
-                           const CUtensorMap&, const pa_cache_desc&, cudaStream_t) {
-  return cudaErrorNotSupported;
+constexpr int kBN = 64;            // keys per tile
+constexpr float kRescaleLog2 = 8.f;
+
+template <int D, int BS, int GH>
+struct PrefillCfg {
+  static constexpr int kTOK = 128 / GH;          // query tokens per tile
+  static constexpr int kHalves = D / 64;         // 128-byte column groups
+  static constexpr int kQBytes = 128 * D * 2;
+  static constexpr int kKBytes = kBN * D * 2;
+  static constexpr int kVBytes = kBN * D * 2;
+  static constexpr int kPBytes = 128 * kBN * 2;
+  static constexpr bool kPInK = kKBytes >= kPBytes;
+  static constexpr int kStageBytes = kKBytes + kVBytes;
+  static constexpr int kNST = 2;
+  static constexpr int kQOff = 0;
+  static constexpr int kStageOff = kQBytes;
+  static constexpr int kPOff = kStageOff + kNST * kStageBytes;
+  static constexpr int kBarOff = kPOff + (kPInK ? 0 : kPBytes);
+  static constexpr int kTmemOff = kBarOff + 8 * 8;
+  static constexpr int kScanOff = kTmemOff + 16;
+  static constexpr int kSeqOff = kScanOff + 32 * 4;
+  static constexpr uint32_t kTmemCols = (kBN + D) <= 128 ? 128 : 256;
+  static constexpr int kBlocksPerTile = kBN / BS;
+  static constexpr uint32_t kIdescS = tc::idesc_bf16_f32(128, kBN, 0, 0);
+  static constexpr uint32_t kIdescO = tc::idesc_bf16_f32(128, D, 0, 1);
+  static size_t smem_bytes(int num_seqs) { return 1024 + kSeqOff + 12ull * (num_seqs + 1); }
+};
+
+__device__ __forceinline__ int prefill_scan(int x, int* warp_tot, int& total) {
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, nw = (blockDim.x + 31) >> 5;
+#pragma unroll
+  for (int off = 1; off < 32; off <<= 1) {
+    const int y = __shfl_up_sync(0xffffffffu, x, off);
+    if (lane >= off) x += y;
+  }
+  if (lane == 31) warp_tot[warp] = x;
+  __syncthreads();
+  if (warp == 0) {
+    int t = lane < nw ? warp_tot[lane] : 0;
+#pragma unroll
+    for (int off = 1; off < 32; off <<= 1) {
+      const int y = __shfl_up_sync(0xffffffffu, t, off);
+      if (lane >= off) t += y;
+    }
+    if (lane < nw) warp_tot[lane] = t;
+  }
+  __syncthreads();
+  total = warp_tot[nw - 1];
+  const int r = x + (warp > 0 ? warp_tot[warp - 1] : 0);
+  __syncthreads();
+  return r;
+}
+
+struct Item {
+  int s, r0, q_len, L, t0, hq0, hk, ntile;
+};
+
+template <int D, int BS, int GH>
+__global__ void __launch_bounds__(160, 2)
+    paged_prefill_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constant__ CUtensorMap kmap,
+                         const __grid_constant__ CUtensorMap vmap, const PrefillArgs a) {
+  using C = PrefillCfg<D, BS, GH>;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint8_t* q_s = smem + C::kQOff;
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::kBarOff);
+  uint64_t* q_full = bars + 0;
+  uint64_t* q_empty = bars + 1;
+  uint64_t* kv_full = bars + 2;   // [2]
+  uint64_t* kv_empty = bars + 4;  // [2]
+  uint64_t* s_done = bars + 6;
+  uint64_t* o_done = bars + 7;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + C::kTmemOff);
+  int* warp_tot = reinterpret_cast<int*>(smem + C::kScanOff);
+  int* prefix = reinterpret_cast<int*>(smem + C::kSeqOff);
+  int* clen = prefix + (a.num_seqs + 1);
+  int* qrow = clen + a.num_seqs;
+
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int G = a.num_q_heads / a.num_kv_heads;
+  const int HGp = a.num_q_heads / GH;  // head groups per tile row set
+
+  if (tid == 0) {
+    mbar_init(q_full, 1);
+    mbar_init(q_empty, 1);
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(&kv_full[i], 1);
+      mbar_init(&kv_empty[i], 1);
+    }
+    mbar_init(s_done, 1);
+    mbar_init(o_done, 1);
+    fence_barrier_init();
+  }
+  if (warp == 0) {
+    tc::tmem_alloc(tmem_slot, C::kTmemCols);
+    tc::tmem_relinquish();
+  }
+  if (warp == 4 && lane == 0) {
+    tma_prefetch_desc(&qmap);
+    tma_prefetch_desc(&kmap);
+    tma_prefetch_desc(&vmap);
+  }
+
+  // ---- tiles of every prefill sequence
+  int carry = 0;
+  if (tid == 0) prefix[0] = 0;
+  for (int base = 0; base < a.num_seqs; base += blockDim.x) {
+    const int s = base + tid;
+    int n = 0;
+    if (s < a.num_seqs) {
+      const int L = __ldg(a.context_lens + s);
+      const int r0 = __ldg(a.query_start_loc + s);
+      const int ql = __ldg(a.query_start_loc + s + 1) - r0;
+      clen[s] = L;
+      qrow[s] = r0;
+      if (ql > 1) {
+        if (L < ql || L > a.max_context_len || L > a.max_blocks_per_seq * BS || r0 < 0 ||
+            r0 + ql > a.num_q_tokens) {
+          raise_flag(a.status, PA_FLAG_CONTEXT_RANGE);
+        } else {
+          n = ((ql + C::kTOK - 1) / C::kTOK) * HGp;
+        }
+      }
+    }
+    int total;
+    const int incl = prefill_scan(n, warp_tot, total);
+    if (s < a.num_seqs) prefix[s + 1] = carry + incl;
+    carry += total;
+  }
+  tc::fence_before_sync();
+  __syncthreads();
+  tc::fence_after_sync();
+  const uint32_t tmem = *tmem_slot;
+  const int W = prefix[a.num_seqs];
+
+  auto item_of = [&](int w) {
+    int lo = 0, hi = a.num_seqs;
+    while (hi - lo > 1) {
+      const int mid = (lo + hi) >> 1;
+      if (prefix[mid] <= w) lo = mid; else hi = mid;
+    }
+    Item it;
+    it.s = lo;
+    const int r = w - prefix[lo];
+    const int mt = r / HGp;
+    const int hg = r - mt * HGp;
+    it.r0 = qrow[lo];
+    it.L = clen[lo];
+    it.q_len = 0;
+    it.t0 = mt * C::kTOK;
+    it.hq0 = hg * GH;
+    it.hk = it.hq0 / G;
+    return it;
+  };
+  auto finish_item = [&](Item& it) {
+    it.q_len = __ldg(a.query_start_loc + it.s + 1) - it.r0;
+    const int t_last = min(it.t0 + C::kTOK, it.q_len) - 1;
+    const int p_max = it.L - it.q_len + t_last;
+    it.ntile = p_max / kBN + 1;
+  };
+
+  if (warp == 4) {
+    // ================= producer
+    if (lane == 0) {
+      uint32_t it_no = 0, gj = 0;
+      for (int w = blockIdx.x; w < W; w += gridDim.x, ++it_no) {
+        Item it = item_of(w);
+        finish_item(it);
+        const int* row = a.block_tables + static_cast<size_t>(it.s) * a.max_blocks_per_seq;
+        const int nblk_valid = (it.L + BS - 1) / BS;
+        mbar_wait(q_empty, (it_no & 1) ^ 1, a.status);
+        mbar_arrive_expect_tx(q_full, C::kQBytes);
+#pragma unroll
+        for (int h = 0; h < C::kHalves; ++h)
+          tma_load_3d(q_s + h * 128 * 128, &qmap, q_full, h * 64, it.hq0, it.r0 + it.t0);
+        for (int j = 0; j < it.ntile; ++j, ++gj) {
+          const uint32_t st = gj & 1;
+          mbar_wait(&kv_empty[st], ((gj >> 1) & 1) ^ 1, a.status);
+          uint8_t* ks = smem + C::kStageOff + st * C::kStageBytes;
+          uint8_t* vs = ks + C::kKBytes;
+          mbar_arrive_expect_tx(&kv_full[st], C::kStageBytes);
+#pragma unroll
+          for (int b = 0; b < C::kBlocksPerTile; ++b) {
+            const int lb = j * C::kBlocksPerTile + b;
+            int phys = -1;
+            if (lb < nblk_valid) {
+              phys = __ldg(row + lb);
+              if (phys < 0 || phys >= a.num_blocks) {
+                raise_flag(a.status, PA_FLAG_BLOCK_RANGE);
+                phys = -1;
+              }
+            }
+#pragma unroll
+            for (int h = 0; h < C::kHalves; ++h) {
+              tma_load_4d(ks + h * kBN * 128 + b * BS * 128, &kmap, &kv_full[st], h * 64, it.hk, 0, phys);
+              tma_load_4d(vs + h * kBN * 128 + b * BS * 128, &vmap, &kv_full[st], h * 64, it.hk, 0, phys);
+            }
+          }
+        }
+      }
+    }
+    return;
+  }
+
+  // ================= warps 0-3: one query row per thread (TMEM lane = row)
+  const int r = tid;
+  const uint32_t t_lane = tmem + (static_cast<uint32_t>(warp * 32) << 16);
+  const uint32_t s_col = 0, o_col = kBN;
+  const uint32_t q_addr = smem_u32(q_s);
+  uint32_t it_no = 0, gj = 0;
+  for (int w = blockIdx.x; w < W; w += gridDim.x, ++it_no) {
+    Item it = item_of(w);
+    finish_item(it);
+    const int tok = it.t0 + r / GH;
+    const int lim = min(it.L - it.q_len + tok, it.L - 1);  // last key this row may see
+    float m_used = -CUDART_INF_F, l = 0.f;
+    mbar_wait(q_full, it_no & 1, a.status);
+    for (int j = 0; j < it.ntile; ++j, ++gj) {
+      const uint32_t st = gj & 1;
+      uint8_t* ks = smem + C::kStageOff + st * C::kStageBytes;
+      uint8_t* vs = ks + C::kKBytes;
+      uint8_t* ps = C::kPInK ? ks : smem + C::kPOff;
+      if (tid == 0) {
+        mbar_wait(&kv_full[st], (gj >> 1) & 1, a.status);
+        tc::fence_after_sync();
+        const uint32_t k_addr = smem_u32(ks);
+#pragma unroll
+        for (int kk = 0; kk < D / 16; ++kk) {
+          const uint32_t off_q = (kk >> 2) * (128 * 128) + (kk & 3) * 32;
+          const uint32_t off_k = (kk >> 2) * (kBN * 128) + (kk & 3) * 32;
+          tc::mma_bf16(tmem + s_col, tc::sw128_desc(q_addr + off_q, 16, 1024),
+                       tc::sw128_desc(k_addr + off_k, 16, 1024), C::kIdescS, kk > 0);
+        }
+        tc::commit(s_done);
+      }
+      __syncwarp();
+      mbar_wait(s_done, gj & 1, a.status);
+      tc::fence_after_sync();
+      float sv[kBN];
+      tc::ld32(t_lane + s_col, sv);
+      tc::ld32(t_lane + s_col + 32, sv + 32);
+      tc::wait_ld();
+      const int kbase = j * kBN;
+      float mx = -CUDART_INF_F;
+#pragma unroll
+      for (int c = 0; c < kBN; ++c) {
+        sv[c] = (kbase + c <= lim) ? sv[c] * a.scale_log2 : -CUDART_INF_F;
+        mx = fmaxf(mx, sv[c]);
+      }
+      // Rescale only when the running max grows by more than 2^8; otherwise
+      // keep the old reference so P stays below 2^8 and O needs no update.
+      const float m_new = fmaxf(m_used, mx);
+      float alpha = 1.f;
+      const bool bump = m_new > m_used + kRescaleLog2;
+      if (bump) {
+        alpha = fast_exp2(m_used - m_new);
+        m_used = m_new;
+      }
+      // s_done(j) also covers every earlier PV MMA, so O is stable here.
+      if (j > 0 && __any_sync(0xffffffffu, bump)) {
+#pragma unroll 1
+        for (int q = 0; q < D / 32; ++q) {
+          float ov[32];
+          tc::ld32(t_lane + o_col + 32 * q, ov);
+          tc::wait_ld();
+#pragma unroll
+          for (int i = 0; i < 32; ++i) ov[i] *= alpha;
+          tc::st32(t_lane + o_col + 32 * q, ov);
+        }
+        tc::wait_st();
+      }
+      l *= alpha;
+      uint8_t* prow = ps + r * 128;
+#pragma unroll
+      for (int c8 = 0; c8 < kBN / 8; ++c8) {
+        uint32_t pk[4];
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+          const float p0 = fast_exp2(sv[c8 * 8 + 2 * i] - m_used);
+          const float p1 = fast_exp2(sv[c8 * 8 + 2 * i + 1] - m_used);
+          l += p0 + p1;
+          const __nv_bfloat162 h2 = __floats2bfloat162_rn(p0, p1);
+          pk[i] = *reinterpret_cast<const uint32_t*>(&h2);
+        }
+        *reinterpret_cast<uint4*>(prow + ((c8 ^ (r & 7)) << 4)) = make_uint4(pk[0], pk[1], pk[2], pk[3]);
+      }
+      // zero V rows at or beyond L (stale tail of the last block)
+      const int vz0 = it.L - kbase;
+      if (vz0 < kBN) {
+        mbar_wait(&kv_full[st], (gj >> 1) & 1, a.status);
+        const int z0 = vz0 > 0 ? vz0 : 0;
+        const int nchunks = (kBN - z0) * C::kHalves * 8;
+        for (int i = tid; i < nchunks; i += 128) {
+          const int h = i / ((kBN - z0) * 8);
+          const int rem = i - h * (kBN - z0) * 8;
+          const int row = z0 + rem / 8, c = rem & 7;
+          *reinterpret_cast<uint4*>(vs + h * kBN * 128 + row * 128 + c * 16) = make_uint4(0, 0, 0, 0);
+        }
+      }
+      fence_proxy_async_smem();
+      tc::fence_before_sync();
+      asm volatile("bar.sync 1, 128;" ::: "memory");
+      if (tid == 0) {
+        tc::fence_after_sync();
+        const uint32_t p_addr = smem_u32(ps), v_addr = smem_u32(vs);
+#pragma unroll
+        for (int kk = 0; kk < kBN / 16; ++kk)
+          tc::mma_bf16(tmem + o_col, tc::sw128_desc(p_addr + kk * 32, 16, 1024),
+                       tc::sw128_desc(v_addr + kk * 16 * 128, kBN * 128, 1024), C::kIdescO, j > 0 || kk > 0);
+        tc::commit(o_done);
+        tc::commit(&kv_empty[st]);
+        if (j == it.ntile - 1) tc::commit(q_empty);
+      }
+      __syncwarp();
+    }
+    // ---- epilogue: O / l -> bf16 rows of this sequence
+    mbar_wait(o_done, (gj - 1) & 1, a.status);
+    tc::fence_after_sync();
+    const float inv_l = 1.f / l;
+    const bool row_ok = tok < it.q_len;
+    __nv_bfloat16* orow = static_cast<__nv_bfloat16*>(a.out) +
+                          (static_cast<size_t>(it.r0 + tok) * a.num_q_heads + it.hq0 + r % GH) * D;
+#pragma unroll 1
+    for (int q = 0; q < D / 32; ++q) {
+      float ov[32];
+      tc::ld32(t_lane + o_col + 32 * q, ov);
+      tc::wait_ld();
+      if (row_ok) {
+#pragma unroll
+        for (int v4 = 0; v4 < 4; ++v4) {
+          uint32_t pk[4];
+#pragma unroll
+          for (int i = 0; i < 4; ++i) {
+            const __nv_bfloat162 h2 =
+                __floats2bfloat162_rn(ov[v4 * 8 + 2 * i] * inv_l, ov[v4 * 8 + 2 * i + 1] * inv_l);
+            pk[i] = *reinterpret_cast<const uint32_t*>(&h2);
+          }
+          *reinterpret_cast<uint4*>(orow + 32 * q + 8 * v4) = make_uint4(pk[0], pk[1], pk[2], pk[3]);
+        }
+      }
+    }
+    tc::fence_before_sync();
+    asm volatile("bar.sync 1, 128;" ::: "memory");
+  }
+  tc::fence_before_sync();
+  asm volatile("bar.sync 1, 128;" ::: "memory");
+  if (warp == 0) tc::tmem_dealloc(tmem, C::kTmemCols);
+}
+
+template <int D, int BS, int GH>
+cudaError_t launch_prefill_t(const PrefillArgs& a, const CUtensorMap& qmap, const CUtensorMap& kmap,
+                             const CUtensorMap& vmap, cudaStream_t stream) {
+  using C = PrefillCfg<D, BS, GH>;
+  auto kern = paged_prefill_kernel<D, BS, GH>;
+  const size_t smem = C::smem_bytes(a.num_seqs);
+  static int configured_smem[64] = {0};
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  if (dev < 64 && configured_smem[dev] < static_cast<int>(smem)) {
+    e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
+    if (e != cudaSuccess) return e;
+    configured_smem[dev] = static_cast<int>(smem);
+  }
+  int per_sm = 0;
+  e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, 160, smem);
+  if (e != cudaSuccess) return e;
+  if (per_sm < 1) return cudaErrorInvalidConfiguration;
+  if (per_sm > 2) per_sm = 2;  // TMEM: 2 x 256 columns per SM
+  const int64_t bound = static_cast<int64_t>(a.num_seqs) * (a.num_q_heads / GH) *
+                        ((a.max_query_len + C::kTOK - 1) / C::kTOK);
+  const int64_t slots = static_cast<int64_t>(num_sms()) * per_sm;
+  const int grid = static_cast<int>(bound < slots ? (bound > 0 ? bound : 1) : slots);
+  kern<<<grid, 160, smem, stream>>>(qmap, kmap, vmap, a);
+  return cudaGetLastError();
+}
+
+template <int D, int BS>
+cudaError_t launch_prefill_gh(const PrefillArgs& a, const CUtensorMap& qmap, const CUtensorMap& kmap,
+                              const CUtensorMap& vmap, int gh, cudaStream_t stream) {
+  switch (gh) {
+    case 16: return launch_prefill_t<D, BS, 16>(a, qmap, kmap, vmap, stream);
+    case 8: return launch_prefill_t<D, BS, 8>(a, qmap, kmap, vmap, stream);
+    case 4: return launch_prefill_t<D, BS, 4>(a, qmap, kmap, vmap, stream);
+    case 2: return launch_prefill_t<D, BS, 2>(a, qmap, kmap, vmap, stream);
+    default: return launch_prefill_t<D, BS, 1>(a, qmap, kmap, vmap, stream);
+  }
+}
+
+template <int D>
+cudaError_t launch_prefill_bs(const PrefillArgs& a, const CUtensorMap& qmap, const CUtensorMap& kmap,
+                              const CUtensorMap& vmap, int bs, int gh, cudaStream_t stream) {
+  switch (bs) {
+    case 8: return launch_prefill_gh<D, 8>(a, qmap, kmap, vmap, gh, stream);
+    case 16: return launch_prefill_gh<D, 16>(a, qmap, kmap, vmap, gh, stream);
+    default: return launch_prefill_gh<D, 32>(a, qmap, kmap, vmap, gh, stream);
+  }
+}
+
+}  // namespace
+
+int32_t prefill_heads_per_tile(int32_t group) {
+  return (group <= 16 && (group & (group - 1)) == 0) ? group : 1;
+}
+
+cudaError_t launch_prefill(const PrefillArgs& a, const CUtensorMap& qmap, const CUtensorMap& kmap,
+                           const CUtensorMap& vmap, const pa_cache_desc& c, cudaStream_t stream) {
+  if (c.dtype != PA_BF16) return cudaErrorNotSupported;
+  const int gh = prefill_heads_per_tile(a.num_q_heads / a.num_kv_heads);
+  if (c.head_dim == 64) return launch_prefill_bs<64>(a, qmap, kmap, vmap, c.block_size, gh, stream);
+  return launch_prefill_bs<128>(a, qmap, kmap, vmap, c.block_size, gh, stream);
 }
 
 }  // namespace pa

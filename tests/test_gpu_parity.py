@@ -159,3 +159,63 @@ def test_repeated_step_is_idempotent(P):
     torch.cuda.synchronize()
     assert torch.equal(first, b.out)
     assert np.array_equal(k0, gs.cache_bits(b.k_cache))
+
+
+# --------------------------------------------------------------------------
+# chunked-prefill rows (tcgen05 path)
+# --------------------------------------------------------------------------
+
+@pytest.mark.parametrize("name", ["mixed_bs8", "mixed_bs16", "mixed_bs32"])
+def test_mixed_config_parity(P, name):
+    wl = W.CONFIGS[name]()
+    b, o, got = _run_both(P, wl)
+    _check_attention(got, o.out, W.BF16, name)
+
+
+def test_mixed_results_agree_across_block_sizes(P):
+    import torch
+    from paged_kv_cache_heads_b200 import scenario as gs
+    outs = []
+    for bs in (8, 16, 32):
+        b = gs.prepare(W.mixed_prefill_decode(bs))
+        gs.run_step(b)
+        torch.cuda.synchronize()
+        outs.append(gs.out_as_f64(b.out, W.BF16))
+        del b
+    assert np.abs(outs[0] - outs[1]).max() < 2e-2 and np.abs(outs[0] - outs[2]).max() < 2e-2
+
+
+def _random_prefill(seed, d, bs, g, hkv=2):
+    q_lens = [2, 37, 130, 1, 64, 1, 200]
+    ctx = [0, 100, 517, 30, 0, 1100, 33]
+    return W.random_case(seed, num_seqs=len(q_lens), q_lens=q_lens, ctx_extra=ctx, num_kv_heads=hkv,
+                         group=g, head_dim=d, block_size=bs, dtype=W.BF16)
+
+
+@pytest.mark.parametrize("d", [64, 128])
+@pytest.mark.parametrize("bs", [8, 16, 32])
+@pytest.mark.parametrize("g", [1, 2, 4, 8, 3])
+def test_random_prefill_sweep(P, d, bs, g):
+    wl = _random_prefill(2000 + d + bs + 11 * g, d, bs, g)
+    b, o, got = _run_both(P, wl)
+    _check_attention(got, o.out, W.BF16, "prefill d=%d bs=%d g=%d" % (d, bs, g))
+
+
+def test_prefill_only_batch_and_full_prompt(P):
+    wl = W.random_case(31, num_seqs=3, q_lens=[256, 129, 33], ctx_extra=[0, 0, 1000], num_kv_heads=8,
+                       group=4, head_dim=128, block_size=16, dtype=W.BF16)
+    b, o, got = _run_both(P, wl)
+    _check_attention(got, o.out, W.BF16, "prefill only")
+
+
+def test_prefill_large_logits_trigger_rescale(P):
+    """Keys scaled so the running max grows tile after tile (exercises the O rescale)."""
+    wl = W.random_case(41, num_seqs=2, q_lens=[96, 40], ctx_extra=[700, 300], num_kv_heads=2, group=4,
+                       head_dim=128, block_size=16, dtype=W.BF16)
+    for op in wl.ops:
+        if op.k is not None and op.k.size:
+            f = W.bf16_bits_to_f32(op.k)
+            ramp = np.linspace(0.5, 6.0, f.shape[0], dtype=np.float32)[:, None, None]
+            op.k = W.f32_to_bf16_bits(f * ramp)
+    b, o, got = _run_both(P, wl)
+    _check_attention(got, o.out, W.BF16, "rescale")
