@@ -164,13 +164,16 @@ def tiny(seed: int = 0) -> Workload:
     return _decode_batch("tiny_paged_decode_fp32", geo, [5, 16, 17, 40], _Draw(seed))
 
 
-def llama7b_decode(seed: int = 0) -> Workload:
+def llama7b_decode(seed: int = 0, num_blocks: int = 8192) -> Workload:
     """32 q = 32 kv heads, head_dim 128, bf16, pool 8192 blocks of 16 (1 GiB per
-    cache), batch 32, L ~ U{128..2048}, blocks from a shuffled free list."""
+    cache), batch 32, L ~ U{128..2048}, blocks from a shuffled free list.
+    ``num_blocks`` shrinks the pool (same lengths and values) for profiling
+    captures that must hold little device memory."""
     draw = _Draw(seed)
-    geo = Geometry(8192, 16, 32, 32, 128, BF16, 128)
+    geo = Geometry(num_blocks, 16, 32, 32, 128, BF16, 128)
     lens = draw.lens.integers(128, 2048, size=32, endpoint=True)
-    return _decode_batch("llama7b_decode_b32_bf16", geo, lens, draw)
+    suffix = "" if num_blocks == 8192 else "_pool%d" % num_blocks
+    return _decode_batch("llama7b_decode_b32_bf16" + suffix, geo, lens, draw)
 
 
 def gqa_long_decode(seed: int = 0) -> Workload:
@@ -276,6 +279,7 @@ def random_case(seed: int, *, num_seqs: int, q_lens, ctx_extra, num_kv_heads: in
 CONFIGS = {
     "tiny": tiny,
     "llama7b": llama7b_decode,
+    "llama7b_pool2560": lambda seed=0: llama7b_decode(seed, 2560),
     "gqa_long": gqa_long_decode,
     "prefix_cow": prefix_cow_decode,
     "mixed_bs8": lambda seed=0: mixed_prefill_decode(8, seed),
