@@ -144,6 +144,35 @@ pa_status pa_attention(const void* q, const void* k_cache, const void* v_cache,
                        size_t workspace_bytes, void* stream);
 
 /*
+ * pa_attention_static_workspace -- pa_attention for callers that cannot
+ * allocate device memory. The pages have no counterpart to this call; it
+ * exists for callers such as a serving process whose device memory is handed
+ * out entirely by its own pool, a plug-in host that does not let a library use
+ * the CUDA allocator, or a latency-critical loop that must avoid cudaMalloc /
+ * cudaFree (they can synchronise the device).
+ *   Arguments and results are those of pa_attention, without the workspace:
+ *   the split-K scratch is a fixed array of PA_STATIC_WORKSPACE_BYTES inside
+ *   this library's device image, held on every GPU that loads the library
+ *   until the process exits. No call allocates or frees anything.
+ *   Batches whose pa_attention_workspace_size() exceeds the array are
+ *   rejected with PA_ERR_UNSUPPORTED (and a message naming both sizes).
+ *   The first call on a device looks up the array's device address
+ *   (cudaGetSymbolAddress) with that device current; make that first call
+ *   before any stream capture.
+ *   All calls on a device share the one array: calls that overlap on the GPU
+ *   (different streams, or different host threads) race on it and must be
+ *   serialised by the caller. Stale contents left by an earlier call are
+ *   never read, so nothing needs clearing between calls.
+ */
+#define PA_STATIC_WORKSPACE_BYTES (16u << 20) /* 16 MiB */
+pa_status pa_attention_static_workspace(const void* q, const void* k_cache, const void* v_cache,
+                                        const int32_t* block_tables, int32_t max_blocks_per_seq,
+                                        const int32_t* context_lens, const int32_t* query_start_loc,
+                                        int32_t num_seqs, int32_t num_q_tokens, int32_t num_q_heads,
+                                        int32_t max_query_len, int32_t max_context_len, float scale,
+                                        const pa_cache_desc* cache, void* out, void* stream);
+
+/*
  * pa_read_device_flags -- read (and optionally clear) the device status word
  * of the current device. Synchronises the device first (all streams).
  *   flags  host out: OR of PA_FLAG_* raised since the last clear

@@ -20,7 +20,7 @@ __all__ = [
     "PAError", "PA_FP32", "PA_BF16", "PA_FLAG_SLOT_RANGE", "PA_FLAG_BLOCK_RANGE",
     "PA_FLAG_CONTEXT_RANGE", "PA_FLAG_PAIR_RANGE", "PA_FLAG_WAIT_TIMEOUT", "CacheDesc",
     "library_path", "load_library", "exported_symbols", "pa_store_kv", "pa_copy_blocks",
-    "pa_attention", "pa_attention_workspace_size", "pa_read_device_flags", "pa_last_error",
+    "pa_attention", "pa_attention_workspace_size", "pa_attention_static_workspace", "pa_read_device_flags", "pa_last_error",
     "pa_version", "BlockManager",
 ]
 
@@ -33,6 +33,7 @@ PA_FLAG_BLOCK_RANGE = 0x2
 PA_FLAG_CONTEXT_RANGE = 0x4
 PA_FLAG_PAIR_RANGE = 0x8
 PA_FLAG_WAIT_TIMEOUT = 0x10
+PA_STATIC_WORKSPACE_BYTES = 16 << 20
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
 
@@ -65,6 +66,8 @@ _SIGNATURES = {
     "pa_attention_workspace_size": (C.c_size_t, [_I32, _I32, _I32, _I32, C.POINTER(CacheDesc)]),
     "pa_attention": (C.c_int, [_P, _P, _P, _P, _I32, _P, _P, _I32, _I32, _I32, _I32, _I32, C.c_float,
                                C.POINTER(CacheDesc), _P, _P, C.c_size_t, _P]),
+    "pa_attention_static_workspace": (C.c_int, [_P, _P, _P, _P, _I32, _P, _P, _I32, _I32, _I32, _I32, _I32,
+                                                 C.c_float, C.POINTER(CacheDesc), _P, _P]),
     "pa_read_device_flags": (C.c_int, [C.POINTER(C.c_uint32), _I32]),
     "pa_last_error": (C.c_char_p, []),
     "pa_version": (C.c_char_p, []),
@@ -188,6 +191,20 @@ def pa_attention(q, k_cache, v_cache, block_tables, max_blocks_per_seq, context_
         _ptr(context_lens), _ptr(query_start_loc), int(num_seqs), int(num_q_tokens), int(num_q_heads),
         int(max_query_len), int(max_context_len), float(scale), C.byref(d), _ptr(out), _ptr(workspace),
         int(workspace_bytes), _stream(stream, q, out)))
+
+
+def pa_attention_static_workspace(q, k_cache, v_cache, block_tables, max_blocks_per_seq, context_lens,
+                                  query_start_loc, num_seqs, num_q_tokens, num_q_heads, max_query_len,
+                                  max_context_len, scale, cache, out, stream=None):
+    """pa_attention without a caller workspace: the split-K scratch is a fixed
+    array inside libpa (PA_STATIC_WORKSPACE_BYTES), for callers that cannot
+    allocate device memory. Calls that overlap on one GPU race on that array."""
+    d = _desc(cache)
+    _check(load_library().pa_attention_static_workspace(
+        _ptr(q), _ptr(k_cache), _ptr(v_cache), _ptr(block_tables), int(max_blocks_per_seq),
+        _ptr(context_lens), _ptr(query_start_loc), int(num_seqs), int(num_q_tokens), int(num_q_heads),
+        int(max_query_len), int(max_context_len), float(scale), C.byref(d), _ptr(out),
+        _stream(stream, q, out)))
 
 
 def pa_read_device_flags(clear: bool = True) -> int:
