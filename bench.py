@@ -289,6 +289,7 @@ def measure_ours(wl, steps: int, warmup: int, device, gpu_index: int):
     barrier()
     torch.cuda.synchronize(device)
     with ClockSampler(gpu_index) as clocks:
+        torch.cuda.nvtx.range_push("pa_timed")   # lets a profiler select the timed steps only
         start.record(stream)
         for i in range(steps):
             gs.run_step(b, attention=False)
@@ -296,6 +297,7 @@ def measure_ours(wl, steps: int, warmup: int, device, gpu_index: int):
             gs.run_attention(b)
             ev[i][1].record(stream)
         end.record(stream)
+        torch.cuda.nvtx.range_pop()
         torch.cuda.synchronize(device)
     barrier()
     ms_total = start.elapsed_time(end)
@@ -329,10 +331,83 @@ def measure_ours(wl, steps: int, warmup: int, device, gpu_index: int):
     torch.cuda.synchronize(device)
     barrier()
     e2e_ms = e0.elapsed_time(e1)
+    kernels = measure_kernels(b)
     flags = P.pa_read_device_flags(clear=True)
-    return dict(ms_total=ms_total, attn_ms=attn_ms, e2e_ms=e2e_ms, h2d=h2d, d2h=d2h, clocks=clocks.summary(),
+    return dict(kernels=kernels, ms_total=ms_total, attn_ms=attn_ms, e2e_ms=e2e_ms, h2d=h2d, d2h=d2h, clocks=clocks.summary(),
                 launches=launches_per_step(b) * steps, step_tokens=b.num_step_tokens,
                 step_pairs=int(b.step_pairs.shape[0]), flags=flags, max_context_len=b.max_context_len)
+
+
+def measure_kernels(b, reps: int = 10):
+    """Side measurements of the other kernels on this workload's caches.
+
+    * store_bulk: one pa_store_kv of every cached token of the batch (their
+      slots, fresh rows) -- the bandwidth-bound bulk fill;
+    * copy: pa_copy_blocks of 256 block pairs (src = a used block, dst = a free one);
+    * prefill_only: pa_attention over the sequences with q_len > 1 alone.
+    Each is timed with CUDA events over ``reps`` back-to-back calls after a warm-up.
+    """
+    import torch
+    import paged_kv_cache_heads_b200 as P
+    from paged_kv_cache_heads_b200 import scenario as gs
+    wl, geo = b.wl, b.wl.geometry
+    dev = b.k_cache.device
+    e = 2 if geo.dtype == "bf16" else 4
+    row = geo.num_kv_heads * geo.head_dim * e
+    res = {}
+
+    def timed(fn):
+        fn()
+        torch.cuda.synchronize(dev)
+        a, z = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record()
+        for _ in range(reps):
+            fn()
+        z.record()
+        torch.cuda.synchronize(dev)
+        return a.elapsed_time(z) / reps
+
+    slots = np.concatenate([np.asarray(s, np.int32) for s in b.host["op_slots"] if len(s)])
+    n = int(slots.size)
+    if n:
+        kk = torch.randint(-2000, 2000, (n, geo.num_kv_heads, geo.head_dim), dtype=torch.int16, device=dev) \
+            if geo.dtype == "bf16" else torch.randn(n, geo.num_kv_heads, geo.head_dim, device=dev)
+        sl = torch.from_numpy(slots).to(dev)
+        kc2, vc2 = torch.empty_like(b.k_cache), torch.empty_like(b.v_cache)
+        ms = timed(lambda: P.pa_store_kv(kk, kk, sl, n, kc2, vc2, b.desc))
+        by = 4 * n * row + 4 * n
+        res["store_bulk"] = {"tokens": n, "launch_ms": ms, "algorithmic_bytes": by, "gbs": by / (ms * 1e-3) / 1e9}
+        del kk, kc2, vc2
+    used = np.unique(b.host["block_tables"][b.host["block_tables"] >= 0])
+    held = set(int(x) for x in used)
+    free = [x for x in range(geo.num_blocks) if x not in held][:256]
+    npairs = min(len(free), len(used), 256)
+    if npairs:
+        pairs = torch.from_numpy(np.stack([used[:npairs], np.asarray(free[:npairs])], 1).astype(np.int32)).to(dev)
+        ms = timed(lambda: P.pa_copy_blocks(pairs, npairs, b.k_cache, b.v_cache, b.desc))
+        by = 4 * npairs * geo.block_size * row
+        res["copy"] = {"pairs": npairs, "launch_ms": ms, "algorithmic_bytes": by, "gbs": by / (ms * 1e-3) / 1e9}
+    pre = [i for i, q in enumerate(wl.q_lens) if q > 1]
+    if pre and pre == list(range(len(pre))):
+        qsl = b.host["query_start_loc"][: len(pre) + 1]
+        t = int(qsl[-1])
+        lens = b.host["context_lens"][: len(pre)]
+        ctx = int(lens.max())
+        mq = int(max(wl.q_lens[i] for i in pre))
+        ws_b = P.pa_attention_workspace_size(len(pre), geo.num_q_heads, mq, ctx, b.desc)
+        ws = torch.empty(max(ws_b, 16), dtype=torch.uint8, device=dev)
+        bt, cl, qs = b.block_tables[: len(pre)].contiguous(), b.context_lens[: len(pre)].contiguous(), \
+            torch.from_numpy(qsl).to(dev)
+        out = torch.empty_like(b.out)
+        ms = timed(lambda: P.pa_attention(b.q, b.k_cache, b.v_cache, bt, geo.max_blocks_per_seq, cl, qs, len(pre),
+                                          t, geo.num_q_heads, mq, ctx, wl.scale, b.desc, out, ws, ws_b))
+        flops = 0
+        for i in pre:
+            L, ql = int(lens[i]), wl.q_lens[i]
+            flops += 4 * geo.head_dim * geo.num_q_heads * sum(L - ql + j + 1 for j in range(ql))
+        res["prefill_only"] = {"seqs": len(pre), "q_tokens": t, "launch_ms": ms, "flops": flops,
+                               "tflops": flops / (ms * 1e-3) / 1e12}
+    return res
 
 
 def workload_config(wl, world: int, l2_note: str):
@@ -423,9 +498,13 @@ def main():
             if peak_src == "measured" else "fallback 6.65 TB/s",
             "algorithmic_bytes_per_launch": work["attn_bytes"], "launch_ms": attn_ms,
             "kv_read_gbs": work["attn_kv_bytes"] / (attn_ms * 1e-3) / 1e9}
-    if work["prefill_flops"]:
-        roof["prefill_flops_per_launch"] = work["prefill_flops"]
-        roof["tensor_frac_of_bf16_peak"] = work["prefill_flops"] / (attn_ms * 1e-3) / 1e12 / bf16_peak
+    kern = r["kernels"]
+    for k in ("store_bulk", "copy"):
+        if k in kern:
+            kern[k]["frac_of_hbm_peak"] = kern[k]["gbs"] / hbm_peak
+    if "prefill_only" in kern:
+        kern["prefill_only"]["frac_of_bf16_peak"] = kern["prefill_only"]["tflops"] / bf16_peak
+        kern["prefill_only"]["peak_tflops"] = bf16_peak
     line = {"metric": METRIC, "value": tokens_all / (ms_step * 1e-3), "unit": UNIT, "n_gpus": world,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": "bf16" if wl.geometry.dtype == "bf16" else "fp32",
@@ -436,6 +515,7 @@ def main():
             "e2e": {"value": tokens_all / (e2e_ms * 1e-3), "unit": UNIT, "h2d_bytes_per_step": r["h2d"],
                     "d2h_bytes_per_step": r["d2h"], "ms_per_step": e2e_ms},
             "gpu_launches": r["launches"], "clocks": r["clocks"], "device_flags": r["flags"],
+            "kernels": kern,
             "step_bytes": work["attn_bytes"] + work["store_bytes"] + work["copy_bytes"]}
     print(json.dumps(line), flush=True)
     return 0

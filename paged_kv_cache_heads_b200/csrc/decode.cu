@@ -141,6 +141,9 @@ __global__ void __launch_bounds__((NCW + 1) * 32)
     tma_prefetch_desc(&kmap);
     tma_prefetch_desc(&vmap);
   }
+  // The split merge (and any prefill grid) may be scheduled now; the merge
+  // waits for this grid's completion before it reads a partial.
+  launch_dependents();
 
   // ---- enumerate the work items of every sequence (decode rows only)
   int carry = 0;
@@ -394,6 +397,8 @@ __global__ void __launch_bounds__((NCW + 1) * 32)
 // One CTA per (sequence, query head): merge the splits of a decode row.
 template <typename T, int D, int BS>
 __global__ void __launch_bounds__(D) decode_combine_kernel(const DecodeArgs a) {
+  launch_dependents();
+  grid_dependency_wait();  // every partial of the decode grid is written
   const int s = blockIdx.x / a.num_q_heads;
   const int h = blockIdx.x - s * a.num_q_heads;
   const int r0 = __ldg(a.query_start_loc + s);
@@ -430,6 +435,8 @@ cudaError_t launch_decode_t(const DecodeArgs& a, const CUtensorMap& kmap, const 
   if (e != cudaSuccess) return e;
   if (dev < 64 && configured_smem[dev] < static_cast<int>(smem)) {
     e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
+    if (e != cudaSuccess) return e;
+    e = cudaFuncSetAttribute(kern, cudaFuncAttributePreferredSharedMemoryCarveout, cudaSharedmemCarveoutMaxShared);
     if (e != cudaSuccess) return e;
     configured_smem[dev] = static_cast<int>(smem);
   }
@@ -469,11 +476,10 @@ template <typename T, int D>
 cudaError_t launch_combine_bs(const DecodeArgs& a, int bs, cudaStream_t stream) {
   const unsigned grid = static_cast<unsigned>(a.num_seqs) * a.num_q_heads;
   switch (bs) {
-    case 8: decode_combine_kernel<T, D, 8><<<grid, D, 0, stream>>>(a); break;
-    case 16: decode_combine_kernel<T, D, 16><<<grid, D, 0, stream>>>(a); break;
-    default: decode_combine_kernel<T, D, 32><<<grid, D, 0, stream>>>(a); break;
+    case 8: return launch_chained(decode_combine_kernel<T, D, 8>, dim3(grid), dim3(D), 0, stream, a);
+    case 16: return launch_chained(decode_combine_kernel<T, D, 16>, dim3(grid), dim3(D), 0, stream, a);
+    default: return launch_chained(decode_combine_kernel<T, D, 32>, dim3(grid), dim3(D), 0, stream, a);
   }
-  return cudaGetLastError();
 }
 
 }  // namespace

@@ -119,6 +119,18 @@ __device__ __forceinline__ void tma_load_3d(void* smem_dst, const CUtensorMap* m
       : "memory");
 }
 
+// ---------------------------------------------------------------- launch chaining
+// Programmatic dependent launch: a kernel launched with programmatic stream
+// serialization may start once every CTA of the previous kernel has executed
+// launch_dependents (or exited); grid_dependency_wait blocks until that
+// previous kernel has completed and its memory is visible.
+__device__ __forceinline__ void launch_dependents() {
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+__device__ __forceinline__ void grid_dependency_wait() {
+  asm volatile("griddepcontrol.wait;" ::: "memory");
+}
+
 // ---------------------------------------------------------------- numerics
 __device__ __forceinline__ float fast_exp2(float x) {
   return exp2f(x);

@@ -73,6 +73,24 @@ cudaError_t launch_prefill(const PrefillArgs& a, const CUtensorMap& qmap, const 
 
 // Query heads packed into one 128-row prefill tile (the rest of its rows are tokens).
 int32_t prefill_heads_per_tile(int32_t group);
+// Launch `kernel` with programmatic stream serialization (it may overlap the
+// tail of the previous kernel on the stream; see griddepcontrol in the kernels).
+template <typename... KArgs, typename... Args>
+cudaError_t launch_chained(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t stream,
+                           Args&&... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kernel, static_cast<Args&&>(args)...);
+}
+
 // Heads of one GQA group handled together by one decode CTA.
 int32_t decode_heads_per_cta(int32_t group);
 // Decode smem stage geometry, used by the launcher and the API's checks.

@@ -379,6 +379,7 @@ __global__ void __launch_bounds__(160, 2)
   tc::fence_before_sync();
   asm volatile("bar.sync 1, 128;" ::: "memory");
   if (warp == 0) tc::tmem_dealloc(tmem, C::kTmemCols);
+  if (tid == 0) grid_dependency_wait();  // finish no earlier than the previous grid
 }
 
 template <int D, int BS, int GH>
@@ -394,6 +395,8 @@ cudaError_t launch_prefill_t(const PrefillArgs& a, const CUtensorMap& qmap, cons
   if (dev < 64 && configured_smem[dev] < static_cast<int>(smem)) {
     e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
     if (e != cudaSuccess) return e;
+    e = cudaFuncSetAttribute(kern, cudaFuncAttributePreferredSharedMemoryCarveout, cudaSharedmemCarveoutMaxShared);
+    if (e != cudaSuccess) return e;
     configured_smem[dev] = static_cast<int>(smem);
   }
   int per_sm = 0;
@@ -405,8 +408,11 @@ cudaError_t launch_prefill_t(const PrefillArgs& a, const CUtensorMap& qmap, cons
                         ((a.max_query_len + C::kTOK - 1) / C::kTOK);
   const int64_t slots = static_cast<int64_t>(num_sms()) * per_sm;
   const int grid = static_cast<int>(bound < slots ? (bound > 0 ? bound : 1) : slots);
-  kern<<<grid, 160, smem, stream>>>(qmap, kmap, vmap, a);
-  return cudaGetLastError();
+  // Chained launch: the prefill rows do not read anything the decode grid
+  // writes, so this grid may start as soon as SMs free up; each CTA waits for
+  // the previous grid before it exits, which keeps stream order for whatever
+  // is launched after pa_attention.
+  return launch_chained(kern, dim3(grid), dim3(160), smem, stream, qmap, kmap, vmap, a);
 }
 
 template <int D, int BS>
