@@ -189,12 +189,9 @@ def step_work(wl, step_tokens: int, step_pairs: int):
 
 
 def launches_per_step(b) -> int:
-    from paged_kv_cache_heads_b200 import pa_attention_workspace_size
-    wl, geo = b.wl, b.wl.geometry
-    n = (1 if b.num_step_tokens else 0) + (1 if b.step_pairs.shape[0] else 0) + 1
-    if pa_attention_workspace_size(len(wl.batch_seqs), geo.num_q_heads, wl.max_query_len, b.max_context_len,
-                                   b.desc) > 0:
-        n += 1
+    """Kernels one step launches: store, copy (if pairs), decode + split merge, prefill (if q_len > 1)."""
+    wl = b.wl
+    n = (1 if b.num_step_tokens else 0) + (1 if b.step_pairs.shape[0] else 0) + 2
     if wl.max_query_len > 1:
         n += 1
     return n

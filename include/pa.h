@@ -100,8 +100,10 @@ pa_status pa_copy_blocks(const int32_t* src_dst_pairs, int32_t num_pairs, void* 
 
 /*
  * pa_attention_workspace_size -- bytes of device workspace pa_attention needs
- * for these sizes (0 when no sequence can be split). Same arguments as the
- * matching pa_attention call. Returns 0 for invalid arguments too; the
+ * for these sizes: per-split partial outputs of decode rows and a small block
+ * prefix; it grows with num_seqs * num_q_heads plus the device's SM count, not
+ * with context length. 0 when num_seqs or max_query_len is 0. Same arguments
+ * as the matching pa_attention call. Returns 0 for invalid arguments too; the
  * matching pa_attention call then reports the error.
  */
 size_t pa_attention_workspace_size(int32_t num_seqs, int32_t num_q_heads, int32_t max_query_len,

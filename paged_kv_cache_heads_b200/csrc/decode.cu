@@ -1,5 +1,5 @@
-// Paged decode attention (query rows with q_len == 1), split-K over the block
-// table with an online softmax, plus the kernel that merges the splits.
+// Paged decode attention (query rows with q_len == 1), split over the block
+// table with an online softmax, plus the kernel that merges split rows.
 //
 // What is computed: for sequence s with L = context_lens[s] keys and query
 // head h, o = softmax(q . K[0:L]^T * scale) . V[0:L], where key i lives in
@@ -8,29 +8,33 @@
 // "vLLM核心架构：PagedAttention原理、KV Cache管理、连续批处理机制",
 // §"一、PagedAttention：虚拟内存的灵感"; the decode call is the one the page
 // "深入解析 nano-vLLM 推理引擎的分页 KV 缓存与内存优化架构",
-// §"工程落地：配置参数与监控指标" hands to a library; that page (§三 of the
-// first) notes decode is bound by memory bandwidth, which shapes this design.
+// §"工程落地：配置参数与监控指标" hands to a library. Decode is bound by memory
+// bandwidth (§"三、连续批处理：让GPU一刻不停" of the first page), which shapes
+// the design.
 //
 // Design (B200):
-//  * Work item = (sequence, group of GH query heads sharing one KV head,
-//    split of the sequence's keys). Splits of one sequence are equal-sized
-//    multiples of the block size, so items are balanced.
-//  * Persistent CTAs (a multiple of the SM count) walk items round-robin.
-//    One producer warp gathers each KV block of the item's KV head with two
-//    TMA tensor loads (K, V: box {D, 1, bs, 1}) into a ring of NST shared
-//    memory stages; the ring keeps running across items, so the HBM stream
-//    never drains between items.
-//  * NCW consumer warps take the ring's blocks round-robin. Within a warp,
-//    LPR lanes hold one 16-byte slice each of a key row (TPW rows per warp
-//    step); q.k is a 16-byte-vector dot product finished with a butterfly
-//    shuffle. Each warp keeps its own running max m, sum l and fp32
-//    accumulator; the warps merge through shared memory at the end of an item.
-//  * GQA: every KV block is read once for the GH query heads of the group.
+//  * A unit is (sequence, group of GH query heads sharing one KV head); its
+//    work is the sequence's ceil(L/bs) KV blocks of that head. All units'
+//    blocks are numbered contiguously (unit-major) and the persistent grid of
+//    G CTAs splits that range evenly: CTA c takes blocks [c*B/G, (c+1)*B/G).
+//    Every CTA streams the same number of blocks, so there is no tail, and a
+//    CTA touches only a few units (segments).
+//  * One producer warp gathers each KV block of the current head with two TMA
+//    tensor loads (K, V: box {D, 1, bs, 1}) into a ring of NST shared-memory
+//    stages; the ring runs on across segments.
+//  * NCW consumer warps take the ring's blocks round-robin. LPR lanes hold one
+//    16-byte slice each of a key row (TPW rows per warp step). q.k uses packed
+//    fp32x2 FMAs; the per-head partial sums are reduce-scattered across the
+//    row's lanes so each lane ends with one head's full score, does that
+//    head's exp, and the lanes exchange probabilities for P.V. Warps merge
+//    their (m, l, acc) through shared memory at the end of a segment.
+//  * GQA: every KV block is read once for the GH query heads of its group.
 //  * Keys at or beyond L (the unfilled tail of the last block) are masked and
 //    their V rows are never read, so stale bits there (even NaN) cannot leak.
-//  * A sequence with one split writes its output rows directly; otherwise
-//    each split writes (o / l, m + log2 l) to the workspace and a second
-//    kernel merges them: O = sum_j 2^(lse_j - M) O_j / sum_j 2^(lse_j - M).
+//  * A unit covered by one CTA writes its output rows directly. Otherwise each
+//    covering CTA c writes (o / l, m + log2 l) to partial slot u + c (unique:
+//    the CTAs covering unit u+1 start where those of unit u end), and a second
+//    kernel merges them: O = sum_c 2^(lse_c - M) O_c / sum_c 2^(lse_c - M).
 #include <math_constants.h>
 
 #include "pa_common.cuh"
@@ -39,16 +43,9 @@
 namespace pa {
 namespace {
 
-// Number of equal splits for a sequence of L keys, and their span (a multiple
-// of the block size, at most chunk tokens).
-__device__ __forceinline__ int split_span(int L, int chunk, int bs) {
-  const int n0 = (L + chunk - 1) / chunk;
-  const int per = (L + n0 - 1) / n0;
-  return ((per + bs - 1) / bs) * bs;
-}
-__device__ __forceinline__ int num_splits(int L, int chunk, int bs) {
-  const int span = split_span(L, chunk, bs);
-  return (L + span - 1) / span;
+// First CTA whose range [c*B/G, (c+1)*B/G) contains block b (0 <= b < B).
+__device__ __forceinline__ int cta_of_block(int64_t b, int64_t B, int G) {
+  return static_cast<int>(((b + 1) * G - 1) / B);
 }
 
 // Block-wide inclusive scan of one int per thread (nthreads <= 1024).
@@ -77,7 +74,10 @@ __device__ __forceinline__ int block_inclusive_scan(int x, int* warp_tot, int& t
   return r;
 }
 
-template <typename T, int D, int BS, int GH, int NCW>
+// KH > 1 (only with GH == 1, KH == NCW): the CTA streams KH adjacent KV heads
+// at once -- one TMA box {D, KH, bs, 1} reads KH*D contiguous elements per
+// token -- and consumer warp w owns head w of every block.
+template <typename T, int D, int BS, int GH, int KH, int NCW>
 struct DecodeCfg {
   static constexpr int kEB = sizeof(T);
   static constexpr int kRowB = D * kEB;             // bytes of one key row (one head)
@@ -85,34 +85,56 @@ struct DecodeCfg {
   static constexpr int kTPW = 32 / kLPR;            // rows per warp step
   static constexpr int kEPL = 16 / kEB;             // elements per lane
   static constexpr int kSteps = BS / kTPW;          // warp steps per block
-  static constexpr int kNIT = kSteps < 8 ? kSteps : 8;  // steps per softmax update
+  static constexpr int kNIT = kSteps < 16 ? kSteps : 16;  // steps per softmax update
   static constexpr int kNUPD = kSteps / kNIT;
-  static constexpr int kStageB = 2 * BS * kRowB;    // K block + V block
-  // Stages: about 64 KiB in flight, and a multiple of NCW so that every use of
-  // a stage belongs to the same consumer warp (its parity waits then never
-  // run more than one phase ahead of the barrier).
+  static constexpr int kLogLPR = kLPR == 32 ? 5 : (kLPR == 16 ? 4 : 3);
+  static constexpr int kLogGH = GH == 4 ? 2 : (GH == 2 ? 1 : 0);
+  static constexpr int kHeadShift = kLogLPR - kLogGH;  // lane bits below the head index
+  static constexpr int kPairs = kEPL / 2;              // fp32 pairs per lane
+  static constexpr int kHPU = GH * KH;                 // query heads per unit
+  static constexpr int kTokB = KH * kRowB;             // bytes per token in a stage
+  static constexpr int kStageB = 2 * BS * kTokB;       // K block + V block
+  // Stages: about 64 KiB in flight per CTA (3 CTAs per SM keep ~192 KiB of
+  // HBM reads outstanding), and a multiple of NCW so that every use of a stage
+  // belongs to the same consumer warp (its parity waits then never run more
+  // than one phase ahead).
+  // With KH > 1 every warp reads every stage, so any count works; ~96 KiB.
   static constexpr int kNST0 = 65536 / kStageB;
   static constexpr int kNST1 = kNST0 < NCW ? NCW : (kNST0 > 16 ? 16 : kNST0);
-  static constexpr int kNST = (kNST1 / NCW) * NCW;
+  static constexpr int kNSTM = 98304 / kStageB;
+  static constexpr int kNST = KH > 1 ? (kNSTM < 2 ? 2 : (kNSTM > 8 ? 8 : kNSTM)) : (kNST1 / NCW) * NCW;
   static constexpr int kThreads = (NCW + 1) * 32;
-  static constexpr int kCombFloats = NCW * GH * (D + 2);
-  // dynamic smem: stages | bars | comb x2 | warp totals | prefix, clen, row
+  static constexpr int kCombFloats = KH > 1 ? 0 : NCW * GH * (D + 2);
+  // dynamic smem: stages | bars | comb | warp totals | abort | seq prefix, clen, row
   static constexpr int kBarOff = kNST * kStageB;
   static constexpr int kCombOff = kBarOff + 2 * kNST * 8;
-  static constexpr int kScanOff = kCombOff + 2 * kCombFloats * 4;
+  static constexpr int kScanOff = kCombOff + kCombFloats * 4;
   static constexpr int kAbortOff = kScanOff + 32 * 4;
   static constexpr int kSeqOff = kAbortOff + 16;
   static_assert(kRowB % 16 == 0 && 32 % kLPR == 0, "row must split into lanes");
   static_assert(BS % kTPW == 0 && kSteps % kNIT == 0, "block must split into steps");
-  static_assert(kNST % NCW == 0, "each stage must always go to the same consumer warp");
+  static_assert(KH > 1 || kNST % NCW == 0, "each stage must always go to the same consumer warp");
+  static_assert(KH == 1 || (GH == 1 && KH == NCW), "multi-head CTAs: one warp per KV head");
+  static_assert(kLogGH <= kLogLPR, "more heads than lanes per row");
   static size_t smem_bytes(int num_seqs) { return 1024 + kSeqOff + 12ull * (num_seqs + 1); }
 };
 
-template <typename T, int D, int BS, int GH, int NCW>
-__global__ void __launch_bounds__((NCW + 1) * 32)
+// One segment: the part of a unit's block range that one CTA streams.
+struct Segment {
+  int s;         // sequence
+  int hg;        // head group (first query head hg * GH)
+  int blo, bhi;  // logical blocks [blo, bhi) of the sequence
+  int L;         // context length
+  int slot;      // partial slot (unit + cta), or -1 when this CTA covers the whole unit
+};
+
+template <typename T, int D, int BS, int GH, int KH, int NCW>
+// Registers are budgeted for 4 (one head) or 3 (grouped heads) CTAs per SM:
+// more resident warps hide the latency of the shuffle and FMA chains.
+__global__ void __launch_bounds__((NCW + 1) * 32, (GH == 1 ? 4 : 3))
     paged_decode_kernel(const __grid_constant__ CUtensorMap kmap,
                         const __grid_constant__ CUtensorMap vmap, const DecodeArgs a) {
-  using C = DecodeCfg<T, D, BS, GH, NCW>;
+  using C = DecodeCfg<T, D, BS, GH, KH, NCW>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint64_t* full = reinterpret_cast<uint64_t*>(smem + C::kBarOff);
@@ -120,19 +142,18 @@ __global__ void __launch_bounds__((NCW + 1) * 32)
   float* comb = reinterpret_cast<float*>(smem + C::kCombOff);
   int* warp_tot = reinterpret_cast<int*>(smem + C::kScanOff);
   volatile int* abort_word = reinterpret_cast<volatile int*>(smem + C::kAbortOff);
-  int* prefix = reinterpret_cast<int*>(smem + C::kSeqOff);      // [S+1]
+  int* prefix = reinterpret_cast<int*>(smem + C::kSeqOff);      // [S+1] decode blocks before seq s
   int* clen = prefix + (a.num_seqs + 1);                         // [S]
   int* qrow = clen + a.num_seqs;                                 // [S]
 
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int G = a.num_q_heads / a.num_kv_heads;
-  const int HG = a.num_q_heads / GH;  // head groups over all KV heads
-  const int chunk = a.chunk_tokens;
+  const int HG = a.num_q_heads / C::kHPU;  // units per sequence
 
   if (tid == 0) {
     for (int i = 0; i < C::kNST; ++i) {
       mbar_init(&full[i], 1);
-      mbar_init(&empty[i], 1);
+      mbar_init(&empty[i], KH > 1 ? NCW : 1);  // KH > 1: every consumer warp releases
     }
     fence_barrier_init();
     *abort_word = 0;
@@ -141,11 +162,11 @@ __global__ void __launch_bounds__((NCW + 1) * 32)
     tma_prefetch_desc(&kmap);
     tma_prefetch_desc(&vmap);
   }
-  // The split merge (and any prefill grid) may be scheduled now; the merge
+  // The merge kernel (and any prefill grid) may be scheduled now; the merge
   // waits for this grid's completion before it reads a partial.
   launch_dependents();
 
-  // ---- enumerate the work items of every sequence (decode rows only)
+  // ---- decode blocks of every sequence, and their prefix
   int carry = 0;
   if (tid == 0) prefix[0] = 0;
   for (int base = 0; base < a.num_seqs; base += blockDim.x) {
@@ -161,7 +182,7 @@ __global__ void __launch_bounds__((NCW + 1) * 32)
         if (L < 1 || L > a.max_context_len || L > a.max_blocks_per_seq * BS) {
           raise_flag(a.status, PA_FLAG_CONTEXT_RANGE);
         } else {
-          n = num_splits(L, chunk, BS) * HG;
+          n = (L + BS - 1) / BS;
         }
       }
     }
@@ -171,48 +192,70 @@ __global__ void __launch_bounds__((NCW + 1) * 32)
     carry += total;
   }
   __syncthreads();
-  const int W = prefix[a.num_seqs];
+  const int64_t B = static_cast<int64_t>(prefix[a.num_seqs]) * HG;  // blocks of all units
+  if (blockIdx.x == 0 && a.seq_prefix)
+    for (int i = tid; i <= a.num_seqs; i += blockDim.x) a.seq_prefix[i] = prefix[i];
+  const int64_t beg = static_cast<int64_t>(blockIdx.x) * B / a.grid;
+  const int64_t end = static_cast<int64_t>(blockIdx.x + 1) * B / a.grid;
 
-  // item -> (sequence, split, head group, key-block range)
-  auto decode_item = [&](int w, int& s, int& j, int& hg, int& blo, int& bhi, int& L) {
-    int lo = 0, hi = a.num_seqs;  // find s: prefix[s] <= w < prefix[s+1]
+  // the segment of this CTA that starts at global block b (beg <= b < end)
+  auto segment_at = [&](int64_t b, Segment& g) {
+    int lo = 0, hi = a.num_seqs;  // largest s with prefix[s] * HG <= b
     while (hi - lo > 1) {
       const int mid = (lo + hi) >> 1;
-      if (prefix[mid] <= w) lo = mid; else hi = mid;
+      if (static_cast<int64_t>(prefix[mid]) * HG <= b) lo = mid; else hi = mid;
     }
-    s = lo;
-    const int r = w - prefix[s];
-    j = r / HG;
-    hg = r - j * HG;
-    L = clen[s];
-    const int span = split_span(L, chunk, BS);
-    const int t0 = j * span;
-    const int t1 = min(t0 + span, L);
-    blo = t0 / BS;
-    bhi = (t1 + BS - 1) / BS;
+    const int nbs = prefix[lo + 1] - prefix[lo];
+    const int64_t off = b - static_cast<int64_t>(prefix[lo]) * HG;
+    const int hg = static_cast<int>(off / nbs);
+    const int lb = static_cast<int>(off - static_cast<int64_t>(hg) * nbs);
+    const int64_t ub0 = b - lb, ub1 = ub0 + nbs;  // the unit's global block range
+    g.s = lo;
+    g.hg = hg;
+    g.blo = lb;
+    g.bhi = lb + static_cast<int>(min(static_cast<int64_t>(nbs - lb), end - b));
+    g.L = clen[lo];
+    g.slot = (ub0 >= beg && ub1 <= end) ? -1 : (lo * HG + hg) + static_cast<int>(blockIdx.x);
   };
 
   if (warp == NCW) {
     // ================= producer warp: TMA gathers of K/V blocks
+    // The block ids of the next segment are fetched while the current
+    // segment's loads are issued, so a segment never waits on a table read.
+    auto fetch_ids = [&](const Segment& g, int b0) {  // raw ids; checked when used
+      return b0 + lane < g.bhi
+                 ? __ldg(a.block_tables + static_cast<size_t>(g.s) * a.max_blocks_per_seq + b0 + lane)
+                 : 0;
+    };
+    auto checked = [&](int phys) {
+      if (phys < 0 || phys >= a.num_blocks) {
+        raise_flag(a.status, PA_FLAG_BLOCK_RANGE);
+        return -1;  // a fully out-of-bounds box: TMA fills zeros, reads nothing
+      }
+      return phys;
+    };
     uint32_t k = 0;
     bool ok = true;
-    for (int w = blockIdx.x; w < W && ok; w += gridDim.x) {
-      int s, j, hg, blo, bhi, L;
-      decode_item(w, s, j, hg, blo, bhi, L);
-      const int hk = (hg * GH) / G;
-      const int* row = a.block_tables + static_cast<size_t>(s) * a.max_blocks_per_seq;
-      for (int b0 = blo; b0 < bhi && ok; b0 += 32) {
-        int phys = -1;
-        if (b0 + lane < bhi) {
-          phys = __ldg(row + b0 + lane);
-          if (phys < 0 || phys >= a.num_blocks) {
-            raise_flag(a.status, PA_FLAG_BLOCK_RANGE);
-            phys = -1;  // a fully out-of-bounds box: TMA fills zeros, reads nothing
-          }
-        }
-        const int cnt = min(32, bhi - b0);
+    Segment cur, nxt;
+    int64_t b = beg;
+    int ids = 0;
+    if (b < end) {
+      segment_at(b, cur);
+      ids = fetch_ids(cur, cur.blo);
+    }
+    while (b < end && ok) {
+      const int64_t bn = b + (cur.bhi - cur.blo);
+      int nids = 0;
+      if (bn < end) {
+        segment_at(bn, nxt);
+        nids = fetch_ids(nxt, nxt.blo);
+      }
+      const int hk = (cur.hg * C::kHPU) / G;  // first KV head of the unit
+      for (int b0 = cur.blo; b0 < cur.bhi && ok; b0 += 32) {
+        int cur_ids = checked(b0 == cur.blo ? ids : fetch_ids(cur, b0));
+        const int cnt = min(32, cur.bhi - b0);
         for (int i = 0; i < cnt; ++i, ++k) {
-          const int pb = __shfl_sync(0xffffffffu, phys, i);
+          const int pb = __shfl_sync(0xffffffffu, cur_ids, i);
           int good = 1;
           if (lane == 0) {
             const uint32_t st = k % C::kNST, use = k / C::kNST;
@@ -221,13 +264,16 @@ __global__ void __launch_bounds__((NCW + 1) * 32)
               uint8_t* dst = smem + st * C::kStageB;
               mbar_arrive_expect_tx(&full[st], C::kStageB);
               tma_load_4d(dst, &kmap, &full[st], 0, hk, 0, pb);
-              tma_load_4d(dst + BS * C::kRowB, &vmap, &full[st], 0, hk, 0, pb);
+              tma_load_4d(dst + BS * C::kTokB, &vmap, &full[st], 0, hk, 0, pb);
             }
           }
           ok = __shfl_sync(0xffffffffu, good, 0) != 0;
           if (!ok) break;
         }
       }
+      cur = nxt;
+      ids = nids;
+      b = bn;
     }
     return;
   }
@@ -236,102 +282,119 @@ __global__ void __launch_bounds__((NCW + 1) * 32)
   const int sub = lane / C::kLPR;  // which row of a warp step
   const int c = lane % C::kLPR;    // which 16-byte slice of the row
   uint32_t k = 0;
-  int item_no = 0;
-  for (int w = blockIdx.x; w < W; w += gridDim.x, ++item_no) {
-    int s, j, hg, blo, bhi, L;
-    decode_item(w, s, j, hg, blo, bhi, L);
-    const int nblk = bhi - blo;
-    const int h0 = hg * GH;
-    const int row = qrow[s];
-
-    float qf[GH][C::kEPL];
+  for (int64_t b = beg; b < end;) {
+    Segment g;
+    segment_at(b, g);
+    b += g.bhi - g.blo;
+    const int blo = g.blo;
+    const int nblk = g.bhi - g.blo;
+    const int h0 = g.hg * C::kHPU + (KH > 1 ? warp : 0);  // first query head of this warp
+    const int row = qrow[g.s];
+    const int L = g.L;
+    // q (pre-multiplied by scale * log2 e) as fp32 pairs for every head of the group
+    float2 q2[GH][C::kPairs];
+    const float2 sc2 = make_float2(a.scale_log2, a.scale_log2);
 #pragma unroll
     for (int g = 0; g < GH; ++g) {
       const uint4 qv = *reinterpret_cast<const uint4*>(
           static_cast<const uint8_t*>(a.q) +
           ((static_cast<size_t>(row) * a.num_q_heads + h0 + g) * D + c * C::kEPL) * C::kEB);
-      Elem<T>::widen(qv, qf[g]);
+      Elem<T>::widen2(qv, q2[g]);
 #pragma unroll
-      for (int e = 0; e < C::kEPL; ++e) qf[g][e] *= a.scale_log2;
+      for (int i = 0; i < C::kPairs; ++i) q2[g][i] = __fmul2_rn(q2[g][i], sc2);
     }
-    float m[GH], l[GH], acc[GH][C::kEPL];
+    // After the reduce-scatter below this lane holds the full score of one
+    // head of the group (hsel); m and l track that head.
+    const int hsel = (c >> C::kHeadShift) & (GH - 1);
+    float m = -CUDART_INF_F, l = 0.f;
+    float2 acc2[GH][C::kPairs];
 #pragma unroll
-    for (int g = 0; g < GH; ++g) {
-      m[g] = -CUDART_INF_F;
-      l[g] = 0.f;
+    for (int g = 0; g < GH; ++g)
 #pragma unroll
-      for (int e = 0; e < C::kEPL; ++e) acc[g][e] = 0.f;
-    }
+      for (int i = 0; i < C::kPairs; ++i) acc2[g][i] = make_float2(0.f, 0.f);
 
     bool ok = true;
-    const int first = (warp - static_cast<int>(k % NCW) + NCW) % NCW;
-    for (int i = first; i < nblk; i += NCW) {
+    const int first = KH > 1 ? 0 : (warp - static_cast<int>(k % NCW) + NCW) % NCW;
+    for (int i = first; i < nblk; i += (KH > 1 ? 1 : NCW)) {
       const uint32_t kk = k + i;
       const uint32_t st = kk % C::kNST;
       if (!mbar_wait(&full[st], (kk / C::kNST) & 1, a.status)) { ok = false; break; }
-      const uint8_t* Ks = smem + st * C::kStageB;
-      const uint8_t* Vs = Ks + BS * C::kRowB;
+      const uint8_t* Ks = smem + st * C::kStageB + (KH > 1 ? warp * C::kRowB : 0);
+      const uint8_t* Vs = Ks + BS * C::kTokB;
       const int tok0 = (blo + i) * BS;
 #pragma unroll
       for (int u = 0; u < C::kNUPD; ++u) {
-        float sc[GH][C::kNIT];
+        float sc[C::kNIT];
 #pragma unroll
         for (int it = 0; it < C::kNIT; ++it) {
           const int t = (u * C::kNIT + it) * C::kTPW + sub;
-          const uint4 kv = *reinterpret_cast<const uint4*>(Ks + t * C::kRowB + c * 16);
-          float kf[C::kEPL];
-          Elem<T>::widen(kv, kf);
+          const uint4 kv = *reinterpret_cast<const uint4*>(Ks + t * C::kTokB + c * 16);
+          float2 k2[C::kPairs];
+          Elem<T>::widen2(kv, k2);
+          float v[GH];
 #pragma unroll
           for (int g = 0; g < GH; ++g) {
-            float p = 0.f;
+            float2 d2 = __fmul2_rn(q2[g][0], k2[0]);
 #pragma unroll
-            for (int e = 0; e < C::kEPL; ++e) p = fmaf(qf[g][e], kf[e], p);
-            sc[g][it] = p;
+            for (int e = 1; e < C::kPairs; ++e) d2 = __ffma2_rn(q2[g][e], k2[e], d2);
+            v[g] = d2.x + d2.y;
           }
+          // reduce-scatter over the head bits of c: each level halves the
+          // heads a lane keeps and adds the partner's half
+#pragma unroll
+          for (int lvl = 0; lvl < C::kLogGH; ++lvl) {
+            const int off = C::kLPR >> (lvl + 1);
+            const bool up = (c & off) != 0;
+            const int half = GH >> (lvl + 1);
+#pragma unroll
+            for (int h = 0; h < half; ++h) {
+              const float keep = up ? v[half + h] : v[h];
+              const float send = up ? v[h] : v[half + h];
+              v[h] = keep + __shfl_xor_sync(0xffffffffu, send, off);
+            }
+          }
+          float s1 = v[0];
+#pragma unroll
+          for (int off = C::kLPR >> (C::kLogGH + 1); off > 0; off >>= 1) s1 += __shfl_xor_sync(0xffffffffu, s1, off);
+          sc[it] = tok0 + t < L ? s1 : -CUDART_INF_F;
         }
+        float mx = sc[0];
+#pragma unroll
+        for (int it = 1; it < C::kNIT; ++it) mx = fmaxf(mx, sc[it]);
+#pragma unroll
+        for (int off = C::kLPR; off < 32; off <<= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, off));
+        const float m_new = fmaxf(m, mx);
+        const float m_use = m_new == -CUDART_INF_F ? 0.f : m_new;
+        const float alpha = fast_exp2(m - m_use);
+        m = m_new;
+        l *= alpha;
 #pragma unroll
         for (int it = 0; it < C::kNIT; ++it) {
-          const bool valid = tok0 + (u * C::kNIT + it) * C::kTPW + sub < L;
-#pragma unroll
-          for (int g = 0; g < GH; ++g) {
-            float p = sc[g][it];
-#pragma unroll
-            for (int off = C::kLPR / 2; off > 0; off >>= 1) p += __shfl_xor_sync(0xffffffffu, p, off);
-            sc[g][it] = valid ? p : -CUDART_INF_F;
-          }
+          const float p = fast_exp2(sc[it] - m_use);
+          sc[it] = p;
+          l += p;
         }
 #pragma unroll
         for (int g = 0; g < GH; ++g) {
-          float mx = sc[g][0];
+          const float ag = GH == 1 ? alpha : __shfl_sync(0xffffffffu, alpha, g << C::kHeadShift);
+          const float2 ag2 = make_float2(ag, ag);
 #pragma unroll
-          for (int it = 1; it < C::kNIT; ++it) mx = fmaxf(mx, sc[g][it]);
-#pragma unroll
-          for (int off = C::kLPR; off < 32; off <<= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, off));
-          const float m_new = fmaxf(m[g], mx);
-          const float m_use = m_new == -CUDART_INF_F ? 0.f : m_new;
-          const float alpha = fast_exp2(m[g] - m_use);
-          m[g] = m_new;
-          l[g] *= alpha;
-#pragma unroll
-          for (int e = 0; e < C::kEPL; ++e) acc[g][e] *= alpha;
-#pragma unroll
-          for (int it = 0; it < C::kNIT; ++it) {
-            const float p = fast_exp2(sc[g][it] - m_use);
-            sc[g][it] = p;
-            l[g] += p;
-          }
+          for (int e = 0; e < C::kPairs; ++e) acc2[g][e] = __fmul2_rn(acc2[g][e], ag2);
         }
 #pragma unroll
         for (int it = 0; it < C::kNIT; ++it) {
           const int t = (u * C::kNIT + it) * C::kTPW + sub;
-          if (tok0 + t < L) {
-            const uint4 vv = *reinterpret_cast<const uint4*>(Vs + t * C::kRowB + c * 16);
-            float vf[C::kEPL];
-            Elem<T>::widen(vv, vf);
+          // rows at or beyond L are never read (stale bits may be NaN); their p is 0
+          const uint4 vv = tok0 + t < L ? *reinterpret_cast<const uint4*>(Vs + t * C::kTokB + c * 16)
+                                        : make_uint4(0u, 0u, 0u, 0u);
+          float2 v2[C::kPairs];
+          Elem<T>::widen2(vv, v2);
 #pragma unroll
-            for (int g = 0; g < GH; ++g)
+          for (int g = 0; g < GH; ++g) {
+            const float pg = GH == 1 ? sc[it] : __shfl_sync(0xffffffffu, sc[it], sub * C::kLPR + (g << C::kHeadShift));
+            const float2 p2 = make_float2(pg, pg);
 #pragma unroll
-              for (int e = 0; e < C::kEPL; ++e) acc[g][e] = fmaf(sc[g][it], vf[e], acc[g][e]);
+            for (int e = 0; e < C::kPairs; ++e) acc2[g][e] = __ffma2_rn(v2[e], p2, acc2[g][e]);
           }
         }
       }
@@ -343,91 +406,167 @@ __global__ void __launch_bounds__((NCW + 1) * 32)
 
     // ---- merge the rows of this warp (lanes with the same slice c)
 #pragma unroll
-    for (int g = 0; g < GH; ++g) {
+    for (int off = C::kLPR; off < 32; off <<= 1) {
+      l += __shfl_xor_sync(0xffffffffu, l, off);
 #pragma unroll
-      for (int off = C::kLPR; off < 32; off <<= 1) {
-        l[g] += __shfl_xor_sync(0xffffffffu, l[g], off);
+      for (int g = 0; g < GH; ++g)
 #pragma unroll
-        for (int e = 0; e < C::kEPL; ++e) acc[g][e] += __shfl_xor_sync(0xffffffffu, acc[g][e], off);
-      }
+        for (int e = 0; e < C::kPairs; ++e) {
+          acc2[g][e].x += __shfl_xor_sync(0xffffffffu, acc2[g][e].x, off);
+          acc2[g][e].y += __shfl_xor_sync(0xffffffffu, acc2[g][e].y, off);
+        }
     }
-    float* cb = comb + (item_no & 1) * C::kCombFloats + warp * GH * (D + 2);
+    if constexpr (KH > 1) {
+      // this warp's head is complete (no other warp saw it): write it
+      if (!ok) return;
+      if (sub == 0) {
+        const float inv_l = 1.f / l;
+        if (g.slot < 0) {
+          T* o = static_cast<T*>(a.out) + (static_cast<size_t>(row) * a.num_q_heads + h0) * D + c * C::kEPL;
+#pragma unroll
+          for (int e = 0; e < C::kPairs; ++e) {
+            o[2 * e] = Elem<T>::narrow(acc2[0][e].x * inv_l);
+            o[2 * e + 1] = Elem<T>::narrow(acc2[0][e].y * inv_l);
+          }
+        } else {
+          const size_t part = static_cast<size_t>(g.slot) * C::kHPU + warp;
+          float* po = a.part_o + part * D + c * C::kEPL;
+#pragma unroll
+          for (int e = 0; e < C::kPairs; ++e) {
+            po[2 * e] = acc2[0][e].x * inv_l;
+            po[2 * e + 1] = acc2[0][e].y * inv_l;
+          }
+          if (c == 0) a.part_lse[part] = m + log2f(l);
+        }
+      }
+      continue;
+    }
+    float* cb = comb + warp * GH * (D + 2);
     if (sub == 0) {
 #pragma unroll
-      for (int g = 0; g < GH; ++g) {
+      for (int g = 0; g < GH; ++g)
 #pragma unroll
-        for (int e = 0; e < C::kEPL; ++e) cb[g * (D + 2) + c * C::kEPL + e] = acc[g][e];
-        if (c == 0) {
-          cb[g * (D + 2) + D] = m[g];
-          cb[g * (D + 2) + D + 1] = l[g];
+        for (int e = 0; e < C::kPairs; ++e) {
+          cb[g * (D + 2) + c * C::kEPL + 2 * e] = acc2[g][e].x;
+          cb[g * (D + 2) + c * C::kEPL + 2 * e + 1] = acc2[g][e].y;
         }
+      if ((c & ((1 << C::kHeadShift) - 1)) == 0) {
+        cb[hsel * (D + 2) + D] = m;
+        cb[hsel * (D + 2) + D + 1] = l;
       }
     }
     asm volatile("bar.sync 1, %0;" ::"r"(NCW * 32) : "memory");
     if (*abort_word) return;  // every consumer warp sees the same value here
 
-    // ---- merge the warps; write the output row or this split's partial
-    const float* cball = comb + (item_no & 1) * C::kCombFloats;
-    const int nsplit = num_splits(L, chunk, BS);
+    // ---- merge the warps; write the output rows or this CTA's partial
+    const float* cball = comb;
     for (int idx = tid; idx < GH * D; idx += NCW * 32) {
-      const int g = idx / D, d = idx - g * D;
+      const int gi = idx / D, d = idx - gi * D;
       float M = -CUDART_INF_F;
 #pragma unroll
-      for (int ww = 0; ww < NCW; ++ww) M = fmaxf(M, cball[(ww * GH + g) * (D + 2) + D]);
+      for (int ww = 0; ww < NCW; ++ww) M = fmaxf(M, cball[(ww * GH + gi) * (D + 2) + D]);
       float sl = 0.f, so = 0.f;
 #pragma unroll
       for (int ww = 0; ww < NCW; ++ww) {
-        const float* pw = cball + (ww * GH + g) * (D + 2);
+        const float* pw = cball + (ww * GH + gi) * (D + 2);
         const float f = fast_exp2(pw[D] - M);
         sl = fmaf(pw[D + 1], f, sl);
         so = fmaf(pw[d], f, so);
       }
       const float o = so / sl;
-      if (nsplit == 1) {
-        static_cast<T*>(a.out)[(static_cast<size_t>(row) * a.num_q_heads + h0 + g) * D + d] = Elem<T>::narrow(o);
+      if (g.slot < 0) {
+        static_cast<T*>(a.out)[(static_cast<size_t>(row) * a.num_q_heads + h0 + gi) * D + d] = Elem<T>::narrow(o);
       } else {
-        const size_t part = (static_cast<size_t>(s) * a.max_splits + j) * a.num_q_heads + h0 + g;
+        const size_t part = static_cast<size_t>(g.slot) * GH + gi;
         a.part_o[part * D + d] = o;
         if (d == 0) a.part_lse[part] = M + log2f(sl);
       }
     }
+    // the merge buffer is reused by the next segment
+    asm volatile("bar.sync 1, %0;" ::"r"(NCW * 32) : "memory");
   }
 }
 
-// One CTA per (sequence, query head): merge the splits of a decode row.
-template <typename T, int D, int BS>
-__global__ void __launch_bounds__(D) decode_combine_kernel(const DecodeArgs a) {
+// One CTA per unit (sequence, head group), GH x D threads: merge the
+// partials of a unit that several CTAs streamed. The weights
+// 2^(lse_c - M) / sum are formed in parallel in shared memory, then each
+// thread sums its (head, column) over the covering CTAs.
+template <typename T, int D, int BS, int GH>  // GH here: query heads per unit
+__global__ void __launch_bounds__(GH * D) decode_combine_kernel(const DecodeArgs a) {
   launch_dependents();
-  grid_dependency_wait();  // every partial of the decode grid is written
-  const int s = blockIdx.x / a.num_q_heads;
-  const int h = blockIdx.x - s * a.num_q_heads;
-  const int r0 = __ldg(a.query_start_loc + s);
-  if (__ldg(a.query_start_loc + s + 1) - r0 != 1) return;
-  const int L = __ldg(a.context_lens + s);
-  if (L < 1 || L > a.max_context_len || L > a.max_blocks_per_seq * BS) return;
-  const int n = num_splits(L, a.chunk_tokens, BS);
-  if (n <= 1) return;
-  const size_t base = static_cast<size_t>(s) * a.max_splits * a.num_q_heads + h;
-  float M = -CUDART_INF_F;
-  for (int j = 0; j < n; ++j) M = fmaxf(M, a.part_lse[base + static_cast<size_t>(j) * a.num_q_heads]);
-  float sw = 0.f, so = 0.f;
-  const int d = threadIdx.x;
-  for (int j = 0; j < n; ++j) {
-    const size_t p = base + static_cast<size_t>(j) * a.num_q_heads;
-    const float w = fast_exp2(a.part_lse[p] - M);
-    sw += w;
-    so = fmaf(w, a.part_o[p * D + d], so);
+  grid_dependency_wait();  // the decode grid (partials and the block prefix) is complete
+  extern __shared__ float wsm[];  // [n][GH] weights, then [GH] max and [GH] sum
+  const int HG = a.num_q_heads / GH;
+  const int u = blockIdx.x;
+  const int s = u / HG, hg = u - s * HG;
+  const int nbs = a.seq_prefix[s + 1] - a.seq_prefix[s];
+  if (nbs == 0) return;
+  const int64_t B = static_cast<int64_t>(a.seq_prefix[a.num_seqs]) * HG;
+  const int64_t ub0 = static_cast<int64_t>(a.seq_prefix[s]) * HG + static_cast<int64_t>(hg) * nbs;
+  const int c0 = cta_of_block(ub0, B, a.grid);
+  const int c1 = cta_of_block(ub0 + nbs - 1, B, a.grid);
+  if (c0 == c1) return;  // one CTA covered the unit and wrote its rows
+  const int n = c1 - c0 + 1;
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  float* mx = wsm + n * GH;
+  float* sm = mx + GH;
+  const size_t slot0 = static_cast<size_t>(u) + c0;
+  // With more CTAs than blocks some CTAs in [c0, c1] stream nothing and wrote
+  // no partial: they get weight 0 (and their slot is never read).
+  auto streams = [&](int cc) {
+    return static_cast<int64_t>(cc) * B / a.grid < static_cast<int64_t>(cc + 1) * B / a.grid;
+  };
+  for (int i = tid; i < n * GH; i += blockDim.x)
+    wsm[i] = streams(c0 + i / GH) ? a.part_lse[slot0 * GH + i] : -CUDART_INF_F;
+  __syncthreads();
+  if (warp < GH) {  // warp g reduces head g over the n partials
+    float m = -CUDART_INF_F;
+    for (int j = lane; j < n; j += 32) m = fmaxf(m, wsm[j * GH + warp]);
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, off));
+    float t = 0.f;
+    for (int j = lane; j < n; j += 32) t += fast_exp2(wsm[j * GH + warp] - m);
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) t += __shfl_xor_sync(0xffffffffu, t, off);
+    if (lane == 0) {
+      mx[warp] = m;
+      sm[warp] = t;
+    }
   }
-  static_cast<T*>(a.out)[(static_cast<size_t>(r0) * a.num_q_heads + h) * D + d] = Elem<T>::narrow(so / sw);
+  __syncthreads();
+  for (int i = tid; i < n * GH; i += blockDim.x) {
+    const int gi = i % GH;
+    wsm[i] = fast_exp2(wsm[i] - mx[gi]) / sm[gi];
+  }
+  __syncthreads();
+  const int gi = tid / D, d = tid - gi * D;
+  const float* po = a.part_o + (slot0 * GH + gi) * D + d;
+  const size_t stride = static_cast<size_t>(GH) * D;
+  float o0 = 0.f, o1 = 0.f, o2 = 0.f, o3 = 0.f;
+  int j = 0;
+  auto term = [&](int jj) {  // weight 0 marks a CTA without a partial: skip its stale slot
+    const float w = wsm[jj * GH + gi];
+    return w != 0.f ? w * po[jj * stride] : 0.f;
+  };
+  for (; j + 4 <= n; j += 4) {
+    o0 += term(j);
+    o1 += term(j + 1);
+    o2 += term(j + 2);
+    o3 += term(j + 3);
+  }
+  for (; j < n; ++j) o0 += term(j);
+  const int row = __ldg(a.query_start_loc + s);
+  static_cast<T*>(a.out)[(static_cast<size_t>(row) * a.num_q_heads + hg * GH + gi) * D + d] =
+      Elem<T>::narrow((o0 + o1) + (o2 + o3));
 }
 
 constexpr int kNCW = 4;
 
-template <typename T, int D, int BS, int GH>
-cudaError_t launch_decode_t(const DecodeArgs& a, const CUtensorMap& kmap, const CUtensorMap& vmap,
+template <typename T, int D, int BS, int GH, int KH>
+cudaError_t launch_decode_t(DecodeArgs& a, const CUtensorMap& kmap, const CUtensorMap& vmap,
                             cudaStream_t stream) {
-  using C = DecodeCfg<T, D, BS, GH, kNCW>;
-  auto kern = paged_decode_kernel<T, D, BS, GH, kNCW>;
+  using C = DecodeCfg<T, D, BS, GH, KH, kNCW>;
+  auto kern = paged_decode_kernel<T, D, BS, GH, KH, kNCW>;
   const size_t smem = C::smem_bytes(a.num_seqs);
   static int configured_smem[64] = {0};
   int dev = 0;
@@ -435,50 +574,72 @@ cudaError_t launch_decode_t(const DecodeArgs& a, const CUtensorMap& kmap, const 
   if (e != cudaSuccess) return e;
   if (dev < 64 && configured_smem[dev] < static_cast<int>(smem)) {
     e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
-    if (e != cudaSuccess) return e;
-    e = cudaFuncSetAttribute(kern, cudaFuncAttributePreferredSharedMemoryCarveout, cudaSharedmemCarveoutMaxShared);
-    if (e != cudaSuccess) return e;
+    if (e == cudaSuccess)
+      e = cudaFuncSetAttribute(kern, cudaFuncAttributePreferredSharedMemoryCarveout, cudaSharedmemCarveoutMaxShared);
+    if (e != cudaSuccess) {
+      (void)cudaGetLastError();  // reported through the return value; do not leave it pending
+      return e;
+    }
     configured_smem[dev] = static_cast<int>(smem);
   }
-  int per_sm = 0;
-  e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, C::kThreads, smem);
-  if (e != cudaSuccess) return e;
-  if (per_sm < 1) return cudaErrorInvalidConfiguration;
-  const int64_t items_bound =
-      static_cast<int64_t>(a.num_seqs) * (a.num_q_heads / GH) * a.max_splits;
-  const int64_t slots = static_cast<int64_t>(num_sms()) * per_sm;
-  const int grid = static_cast<int>(items_bound < slots ? (items_bound > 0 ? items_bound : 1) : slots);
+  const int per_sm = ctas_per_sm(reinterpret_cast<const void*>(kern), C::kThreads, smem, 8);
+  int grid = num_sms() * per_sm;
+  if (grid > decode_max_grid()) grid = decode_max_grid();
+  if (const char* env = getenv("PA_DECODE_GRID")) {  // testing / tuning: cap the grid
+    const int v = atoi(env);
+    if (v >= 1 && v < grid) grid = v;
+  }
+  a.grid = grid;
+  log_launch("paged_decode_kernel", grid, C::kThreads, smem, per_sm);
   kern<<<grid, C::kThreads, smem, stream>>>(kmap, vmap, a);
   return cudaGetLastError();
 }
 
 template <typename T, int D, int BS>
-cudaError_t launch_decode_gh(const DecodeArgs& a, const CUtensorMap& kmap, const CUtensorMap& vmap,
-                             cudaStream_t stream) {
-  switch (decode_heads_per_cta(a.num_q_heads / a.num_kv_heads)) {
-    case 4: return launch_decode_t<T, D, BS, 4>(a, kmap, vmap, stream);
-    case 2: return launch_decode_t<T, D, BS, 2>(a, kmap, vmap, stream);
-    default: return launch_decode_t<T, D, BS, 1>(a, kmap, vmap, stream);
+cudaError_t launch_decode_gh(DecodeArgs& a, const CUtensorMap& kmap, const CUtensorMap& vmap,
+                             const pa_cache_desc& desc, cudaStream_t stream) {
+  const int group = a.num_q_heads / a.num_kv_heads;
+  if (decode_kv_heads_per_cta(group, desc) == kNCW) return launch_decode_t<T, D, BS, 1, kNCW>(a, kmap, vmap, stream);
+  switch (decode_heads_per_cta(group)) {
+    case 4: return launch_decode_t<T, D, BS, 4, 1>(a, kmap, vmap, stream);
+    case 2: return launch_decode_t<T, D, BS, 2, 1>(a, kmap, vmap, stream);
+    default: return launch_decode_t<T, D, BS, 1, 1>(a, kmap, vmap, stream);
   }
 }
 
 template <typename T, int D>
-cudaError_t launch_decode_bs(const DecodeArgs& a, const CUtensorMap& kmap, const CUtensorMap& vmap,
-                             int bs, cudaStream_t stream) {
-  switch (bs) {
-    case 8: return launch_decode_gh<T, D, 8>(a, kmap, vmap, stream);
-    case 16: return launch_decode_gh<T, D, 16>(a, kmap, vmap, stream);
-    default: return launch_decode_gh<T, D, 32>(a, kmap, vmap, stream);
+cudaError_t launch_decode_bs(DecodeArgs& a, const CUtensorMap& kmap, const CUtensorMap& vmap,
+                             const pa_cache_desc& desc, cudaStream_t stream) {
+  switch (desc.block_size) {
+    case 8: return launch_decode_gh<T, D, 8>(a, kmap, vmap, desc, stream);
+    case 16: return launch_decode_gh<T, D, 16>(a, kmap, vmap, desc, stream);
+    default: return launch_decode_gh<T, D, 32>(a, kmap, vmap, desc, stream);
+  }
+}
+
+template <typename T, int D, int BS, int GH>
+cudaError_t launch_combine_t(const DecodeArgs& a, cudaStream_t stream) {
+  auto kern = decode_combine_kernel<T, D, BS, GH>;
+  const size_t smem = (static_cast<size_t>(a.grid) + 2) * GH * sizeof(float);
+  const unsigned grid = static_cast<unsigned>(a.num_seqs) * (a.num_q_heads / GH);
+  return launch_chained(kern, dim3(grid), dim3(GH * D), smem, stream, a);
+}
+
+template <typename T, int D, int BS>
+cudaError_t launch_combine_gh(const DecodeArgs& a, const pa_cache_desc& desc, cudaStream_t stream) {
+  switch (decode_heads_per_unit(a.num_q_heads / a.num_kv_heads, desc)) {
+    case 4: return launch_combine_t<T, D, BS, 4>(a, stream);
+    case 2: return launch_combine_t<T, D, BS, 2>(a, stream);
+    default: return launch_combine_t<T, D, BS, 1>(a, stream);
   }
 }
 
 template <typename T, int D>
-cudaError_t launch_combine_bs(const DecodeArgs& a, int bs, cudaStream_t stream) {
-  const unsigned grid = static_cast<unsigned>(a.num_seqs) * a.num_q_heads;
-  switch (bs) {
-    case 8: return launch_chained(decode_combine_kernel<T, D, 8>, dim3(grid), dim3(D), 0, stream, a);
-    case 16: return launch_chained(decode_combine_kernel<T, D, 16>, dim3(grid), dim3(D), 0, stream, a);
-    default: return launch_chained(decode_combine_kernel<T, D, 32>, dim3(grid), dim3(D), 0, stream, a);
+cudaError_t launch_combine_bs(const DecodeArgs& a, const pa_cache_desc& desc, cudaStream_t stream) {
+  switch (desc.block_size) {
+    case 8: return launch_combine_gh<T, D, 8>(a, desc, stream);
+    case 16: return launch_combine_gh<T, D, 16>(a, desc, stream);
+    default: return launch_combine_gh<T, D, 32>(a, desc, stream);
   }
 }
 
@@ -490,44 +651,36 @@ int32_t decode_heads_per_cta(int32_t group) {
   return 1;
 }
 
-cudaError_t launch_decode(const DecodeArgs& a, const CUtensorMap& kmap, const CUtensorMap& vmap,
+int32_t decode_kv_heads_per_cta(int32_t group, const pa_cache_desc& c) {
+  // 4 adjacent KV heads per CTA when there is no grouping, the heads divide
+  // evenly, and two 4-head stages (K + V) fit in 128 KiB of shared memory.
+  const int64_t stage = 2ll * c.block_size * kNCW * c.head_dim * (c.dtype == PA_BF16 ? 2 : 4);
+  return (group == 1 && c.num_kv_heads % kNCW == 0 && stage <= 65536) ? kNCW : 1;
+}
+
+int32_t decode_heads_per_unit(int32_t group, const pa_cache_desc& c) {
+  return decode_heads_per_cta(group) * decode_kv_heads_per_cta(group, c);
+}
+
+int32_t decode_max_grid() { return num_sms() * 8; }
+
+cudaError_t launch_decode(DecodeArgs& a, const CUtensorMap& kmap, const CUtensorMap& vmap,
                           const pa_cache_desc& c, cudaStream_t stream) {
   if (c.dtype == PA_BF16) {
-    if (c.head_dim == 64) return launch_decode_bs<__nv_bfloat16, 64>(a, kmap, vmap, c.block_size, stream);
-    return launch_decode_bs<__nv_bfloat16, 128>(a, kmap, vmap, c.block_size, stream);
+    if (c.head_dim == 64) return launch_decode_bs<__nv_bfloat16, 64>(a, kmap, vmap, c, stream);
+    return launch_decode_bs<__nv_bfloat16, 128>(a, kmap, vmap, c, stream);
   }
-  if (c.head_dim == 64) return launch_decode_bs<float, 64>(a, kmap, vmap, c.block_size, stream);
-  return launch_decode_bs<float, 128>(a, kmap, vmap, c.block_size, stream);
+  if (c.head_dim == 64) return launch_decode_bs<float, 64>(a, kmap, vmap, c, stream);
+  return launch_decode_bs<float, 128>(a, kmap, vmap, c, stream);
 }
 
 cudaError_t launch_decode_combine(const DecodeArgs& a, const pa_cache_desc& c, cudaStream_t stream) {
   if (c.dtype == PA_BF16) {
-    if (c.head_dim == 64) return launch_combine_bs<__nv_bfloat16, 64>(a, c.block_size, stream);
-    return launch_combine_bs<__nv_bfloat16, 128>(a, c.block_size, stream);
+    if (c.head_dim == 64) return launch_combine_bs<__nv_bfloat16, 64>(a, c, stream);
+    return launch_combine_bs<__nv_bfloat16, 128>(a, c, stream);
   }
-  if (c.head_dim == 64) return launch_combine_bs<float, 64>(a, c.block_size, stream);
-  return launch_combine_bs<float, 128>(a, c.block_size, stream);
-}
-
-int32_t decode_chunk_tokens(int32_t num_seqs, int32_t num_kv_heads, int32_t group,
-                            int32_t max_context_len, int32_t block_size) {
-  // Aim for several items per resident CTA slot so the round-robin tail is
-  // short, assuming the average sequence is half the longest one; never split
-  // finer than 4 blocks or coarser than 512 tokens.
-  const int64_t units = static_cast<int64_t>(num_seqs) * num_kv_heads *
-                        (group / decode_heads_per_cta(group));
-  const int64_t target_items = 8ll * 148 * 2;
-  const int64_t avg_tokens = max_context_len > 1 ? max_context_len / 2 : 1;
-  int64_t chunk = units > 0 ? (units * avg_tokens + target_items - 1) / target_items : 512;
-  const int64_t lo = 4ll * block_size;
-  if (chunk < lo) chunk = lo;
-  if (chunk > 512) chunk = 512;
-  chunk = ((chunk + block_size - 1) / block_size) * block_size;
-  if (const char* env = getenv("PA_DECODE_CHUNK")) {
-    const int64_t v = atoll(env);
-    if (v >= block_size) chunk = (v / block_size) * block_size;
-  }
-  return static_cast<int32_t>(chunk);
+  if (c.head_dim == 64) return launch_combine_bs<float, 64>(a, c, stream);
+  return launch_combine_bs<float, 128>(a, c, stream);
 }
 
 }  // namespace pa

@@ -135,15 +135,16 @@ pa_status tensor_map(CUtensorMap* out, const void* base, int rank, const uint64_
   return PA_OK;
 }
 
-// Cache as a 4-D tensor {head_dim, num_kv_heads, block_size, num_blocks}.
+// Cache as a 4-D tensor {head_dim, num_kv_heads, block_size, num_blocks}; the
+// box is {box_d, box_heads, block_size, 1}: one block of box_heads adjacent heads.
 pa_status cache_map(CUtensorMap* out, const void* cache, const pa_cache_desc& c, uint32_t box_d,
-                    int swizzle) {
+                    int swizzle, uint32_t box_heads = 1) {
   const uint64_t eb = c.dtype == PA_BF16 ? 2 : 4;
   const uint64_t dims[4] = {uint64_t(c.head_dim), uint64_t(c.num_kv_heads), uint64_t(c.block_size),
                             uint64_t(c.num_blocks)};
   const uint64_t strides[3] = {c.head_dim * eb, uint64_t(c.num_kv_heads) * c.head_dim * eb,
                                uint64_t(c.block_size) * c.num_kv_heads * c.head_dim * eb};
-  const uint32_t box[4] = {box_d, 1, uint32_t(c.block_size), 1};
+  const uint32_t box[4] = {box_d, box_heads, uint32_t(c.block_size), 1};
   return tensor_map(out, cache, 4, dims, strides, box, c.dtype, swizzle);
 }
 
@@ -174,6 +175,39 @@ constexpr int32_t kMaxSeqs = 8192;
 }  // namespace
 
 void set_last_error(const char* msg) { g_last_error = msg; }
+
+int32_t ctas_per_sm(const void* kernel, int threads, size_t smem, int cap) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return 1;
+  int smem_sm = 0, reserved = 0, regs_sm = 0, max_threads = 0;
+  cudaDeviceGetAttribute(&smem_sm, cudaDevAttrMaxSharedMemoryPerMultiprocessor, dev);
+  cudaDeviceGetAttribute(&reserved, cudaDevAttrReservedSharedMemoryPerBlock, dev);
+  cudaDeviceGetAttribute(&regs_sm, cudaDevAttrMaxRegistersPerMultiprocessor, dev);
+  cudaDeviceGetAttribute(&max_threads, cudaDevAttrMaxThreadsPerMultiProcessor, dev);
+  cudaFuncAttributes fa;
+  if (cudaFuncGetAttributes(&fa, kernel) != cudaSuccess) return 1;
+  const int warps = (threads + 31) / 32;
+  const int regs_warp = ((fa.numRegs * 32 + 255) / 256) * 256;  // allocation unit: 256 per warp
+  int n = cap;
+  if (smem + fa.sharedSizeBytes > 0) {
+    const int by_smem = smem_sm / static_cast<int>(smem + fa.sharedSizeBytes + reserved);
+    if (by_smem < n) n = by_smem;
+  }
+  if (regs_warp > 0) {
+    const int by_regs = regs_sm / (regs_warp * warps);
+    if (by_regs < n) n = by_regs;
+  }
+  if (max_threads / threads < n) n = max_threads / threads;
+  return n < 1 ? 1 : n;
+}
+
+void log_launch(const char* kernel, int grid, int block, size_t smem, int per_sm) {
+  static const bool on = [] {
+    const char* e = getenv("PA_LOG_LAUNCH");
+    return e && e[0] == '1';
+  }();
+  if (on) fprintf(stderr, "[libpa] %s grid=%d block=%d smem=%zu ctas/sm=%d\n", kernel, grid, block, smem, per_sm);
+}
 
 int32_t num_sms() {
   static int cache[kMaxDevices] = {0};
@@ -241,33 +275,34 @@ pa_status pa_copy_blocks(const int32_t* src_dst_pairs, int32_t num_pairs, void* 
 }
 
 namespace {
-// Split geometry of one call, or false for arguments the size query cannot use.
-bool split_geometry(int32_t num_seqs, int32_t num_q_heads, int32_t max_query_len,
-                    int32_t max_context_len, const pa_cache_desc* cache, int32_t* chunk,
-                    int32_t* max_splits, size_t* bytes, size_t* lse_offset) {
-  if (!cache || check_cache(cache) != PA_OK || num_seqs < 0 || num_q_heads < 1 ||
-      max_query_len < 0 || max_context_len < 0 || num_q_heads % cache->num_kv_heads)
+// Workspace layout of one call: partial outputs, their log-sum-exp, and the
+// per-sequence decode block prefix. False for arguments the size query cannot use.
+struct WorkspaceLayout {
+  size_t bytes = 0, lse_off = 0, prefix_off = 0;
+};
+bool workspace_layout(int32_t num_seqs, int32_t num_q_heads, int32_t max_query_len, int32_t max_context_len,
+                      const pa_cache_desc* cache, WorkspaceLayout* w) {
+  if (!cache || check_cache(cache) != PA_OK || num_seqs < 0 || num_q_heads < 1 || max_query_len < 0 ||
+      max_context_len < 0 || num_q_heads % cache->num_kv_heads)
     return false;
-  const int32_t g = num_q_heads / cache->num_kv_heads;
-  *chunk = decode_chunk_tokens(num_seqs, cache->num_kv_heads, g, max_context_len, cache->block_size);
-  *max_splits = max_context_len > 0 ? ceil_div(max_context_len, *chunk) : 1;
-  *bytes = 0;
-  *lse_offset = 0;
-  if (max_query_len < 1 || *max_splits <= 1 || num_seqs == 0) return true;
-  const size_t parts = size_t(num_seqs) * *max_splits * num_q_heads;
-  *lse_offset = (parts * cache->head_dim * 4 + 255) & ~size_t(255);
-  *bytes = *lse_offset + parts * 4;
+  *w = WorkspaceLayout();
+  if (max_query_len < 1 || num_seqs == 0) return true;
+  const int32_t gh = decode_heads_per_unit(num_q_heads / cache->num_kv_heads, *cache);
+  // partial slot u + c for unit u = (sequence, head group) and covering CTA c
+  const size_t slots = size_t(num_seqs) * (num_q_heads / gh) + size_t(decode_max_grid());
+  const size_t parts = slots * gh;
+  w->lse_off = (parts * cache->head_dim * 4 + 255) & ~size_t(255);
+  w->prefix_off = (w->lse_off + parts * 4 + 255) & ~size_t(255);
+  w->bytes = w->prefix_off + (size_t(num_seqs) + 1) * 4;
   return true;
 }
 }  // namespace
 
 size_t pa_attention_workspace_size(int32_t num_seqs, int32_t num_q_heads, int32_t max_query_len,
                                    int32_t max_context_len, const pa_cache_desc* cache) {
-  int32_t chunk, ms;
-  size_t bytes, off;
-  if (!split_geometry(num_seqs, num_q_heads, max_query_len, max_context_len, cache, &chunk, &ms, &bytes, &off))
-    return 0;
-  return bytes;
+  WorkspaceLayout w;
+  if (!workspace_layout(num_seqs, num_q_heads, max_query_len, max_context_len, cache, &w)) return 0;
+  return w.bytes;
 }
 
 pa_status pa_attention(const void* q, const void* k_cache, const void* v_cache,
@@ -299,10 +334,9 @@ pa_status pa_attention(const void* q, const void* k_cache, const void* v_cache,
     return fail(PA_ERR_UNSUPPORTED, "query rows with q_len > 1 need a bf16 cache");
   if (!(scale == scale)) return fail(PA_ERR_INVALID_ARG, "scale is NaN");
 
-  int32_t chunk, max_splits;
-  size_t need, lse_off;
-  split_geometry(num_seqs, num_q_heads, max_query_len, max_context_len, cache, &chunk, &max_splits,
-                 &need, &lse_off);
+  WorkspaceLayout wl;
+  workspace_layout(num_seqs, num_q_heads, max_query_len, max_context_len, cache, &wl);
+  const size_t need = wl.bytes;
   if (need > 0 && (!workspace || workspace_bytes < need))
     return fail(PA_ERR_INVALID_ARG, "workspace of %zu bytes needed, %zu given", need,
                 workspace ? workspace_bytes : size_t(0));
@@ -321,8 +355,9 @@ pa_status pa_attention(const void* q, const void* k_cache, const void* v_cache,
   a.block_tables = block_tables;
   a.context_lens = context_lens;
   a.query_start_loc = query_start_loc;
-  a.part_o = need ? static_cast<float*>(workspace) : nullptr;
-  a.part_lse = need ? reinterpret_cast<float*>(static_cast<char*>(workspace) + lse_off) : nullptr;
+  a.part_o = static_cast<float*>(workspace);
+  a.part_lse = reinterpret_cast<float*>(static_cast<char*>(workspace) + wl.lse_off);
+  a.seq_prefix = reinterpret_cast<int32_t*>(static_cast<char*>(workspace) + wl.prefix_off);
   a.status = status;
   a.max_blocks_per_seq = max_blocks_per_seq;
   a.num_seqs = num_seqs;
@@ -330,19 +365,17 @@ pa_status pa_attention(const void* q, const void* k_cache, const void* v_cache,
   a.num_kv_heads = cache->num_kv_heads;
   a.num_blocks = cache->num_blocks;
   a.max_context_len = max_context_len;
-  a.chunk_tokens = chunk;
-  a.max_splits = max_splits;
+  a.grid = 0;
   a.scale_log2 = scale_log2;
 
   CUtensorMap kmap, vmap;
-  if ((st = cache_map(&kmap, k_cache, *cache, cache->head_dim, 0)) != PA_OK) return st;
-  if ((st = cache_map(&vmap, v_cache, *cache, cache->head_dim, 0)) != PA_OK) return st;
+  const uint32_t kh = decode_kv_heads_per_cta(num_q_heads / cache->num_kv_heads, *cache);
+  if ((st = cache_map(&kmap, k_cache, *cache, cache->head_dim, 0, kh)) != PA_OK) return st;
+  if ((st = cache_map(&vmap, v_cache, *cache, cache->head_dim, 0, kh)) != PA_OK) return st;
   e = launch_decode(a, kmap, vmap, *cache, s);
   if (e != cudaSuccess) return cuda_fail(e, "decode launch");
-  if (max_splits > 1) {
-    e = launch_decode_combine(a, *cache, s);
-    if (e != cudaSuccess) return cuda_fail(e, "decode combine launch");
-  }
+  e = launch_decode_combine(a, *cache, s);
+  if (e != cudaSuccess) return cuda_fail(e, "decode combine launch");
   if (max_query_len > 1) {
     PrefillArgs p;
     p.out = out;

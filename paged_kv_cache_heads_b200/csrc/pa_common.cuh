@@ -162,6 +162,12 @@ template <>
 struct Elem<__nv_bfloat16> {
   static constexpr int kPerVec = 8;
   __device__ __forceinline__ static void widen(const uint4& v, float* f) { bf16x8_to_f32(v, f); }
+  // the 8 values as 4 (even, odd) fp32 pairs, for packed f32x2 arithmetic
+  __device__ __forceinline__ static void widen2(const uint4& v, float2* f) {
+    const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+    for (int i = 0; i < 4; ++i) f[i] = make_float2(__uint_as_float(w[i] << 16), __uint_as_float(w[i] & 0xFFFF0000u));
+  }
   __device__ __forceinline__ static __nv_bfloat16 narrow(float x) { return __float2bfloat16_rn(x); }
 };
 
@@ -169,6 +175,10 @@ template <>
 struct Elem<float> {
   static constexpr int kPerVec = 4;
   __device__ __forceinline__ static void widen(const uint4& v, float* f) { f32x4_from_u4(v, f); }
+  __device__ __forceinline__ static void widen2(const uint4& v, float2* f) {
+    f[0] = make_float2(__uint_as_float(v.x), __uint_as_float(v.y));
+    f[1] = make_float2(__uint_as_float(v.z), __uint_as_float(v.w));
+  }
   __device__ __forceinline__ static float narrow(float x) { return x; }
 };
 

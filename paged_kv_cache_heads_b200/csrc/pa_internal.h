@@ -18,18 +18,18 @@ struct DecodeArgs {
   const int32_t* block_tables;
   const int32_t* context_lens;
   const int32_t* query_start_loc;
-  float* part_o;     // [num_seqs][max_splits][num_q_heads][head_dim] fp32 (or null)
-  float* part_lse;   // [num_seqs][max_splits][num_q_heads] fp32, log2 domain (or null)
-  unsigned* status;  // library status word
+  float* part_o;        // [slots][GH][head_dim] fp32 partial outputs
+  float* part_lse;      // [slots][GH] fp32 log2-sum-exp of each partial
+  int32_t* seq_prefix;  // [num_seqs + 1] decode blocks before each sequence
+  unsigned* status;     // library status word
   int32_t max_blocks_per_seq;
   int32_t num_seqs;
   int32_t num_q_heads;
   int32_t num_kv_heads;
   int32_t num_blocks;
   int32_t max_context_len;
-  int32_t chunk_tokens;  // upper bound on keys per split (multiple of block_size)
-  int32_t max_splits;    // ceil(max_context_len / chunk_tokens)
-  float scale_log2;      // scale * log2(e)
+  int32_t grid;         // CTAs of the decode grid (set by launch_decode)
+  float scale_log2;     // scale * log2(e)
 };
 
 struct PrefillArgs {
@@ -52,9 +52,8 @@ struct PrefillArgs {
 // Sets the calling thread's pa_last_error() message.
 void set_last_error(const char* msg);
 
-// Split policy shared by the workspace size query and the launch.
-int32_t decode_chunk_tokens(int32_t num_seqs, int32_t num_kv_heads, int32_t group,
-                            int32_t max_context_len, int32_t block_size);
+// Upper bound on the decode grid; the workspace holds S*Hq/GH + this many partial slots.
+int32_t decode_max_grid();
 inline int32_t ceil_div(int64_t a, int64_t b) { return static_cast<int32_t>((a + b - 1) / b); }
 
 // Launchers return cudaSuccess or the launch error. `maps` are encoded tensor
@@ -65,7 +64,7 @@ cudaError_t launch_store_kv(const void* k, const void* v, const int32_t* slots, 
 cudaError_t launch_copy_blocks(const int32_t* pairs, int32_t num_pairs, void* k_cache,
                                void* v_cache, const pa_cache_desc& c, unsigned* status,
                                cudaStream_t stream);
-cudaError_t launch_decode(const DecodeArgs& a, const CUtensorMap& kmap, const CUtensorMap& vmap,
+cudaError_t launch_decode(DecodeArgs& a, const CUtensorMap& kmap, const CUtensorMap& vmap,
                           const pa_cache_desc& c, cudaStream_t stream);
 cudaError_t launch_decode_combine(const DecodeArgs& a, const pa_cache_desc& c, cudaStream_t stream);
 cudaError_t launch_prefill(const PrefillArgs& a, const CUtensorMap& qmap, const CUtensorMap& kmap,
@@ -91,6 +90,17 @@ cudaError_t launch_chained(void (*kernel)(KArgs...), dim3 grid, dim3 block, size
   return cudaLaunchKernelEx(&cfg, kernel, static_cast<Args&&>(args)...);
 }
 
+// Resident CTAs per SM for a kernel using `smem` dynamic shared memory, from
+// the device's shared-memory and register limits (and `cap`).
+int32_t ctas_per_sm(const void* kernel, int threads, size_t smem, int cap);
+
+// Opt-in launch trace on stderr (environment PA_LOG_LAUNCH=1).
+void log_launch(const char* kernel, int grid, int block, size_t smem, int per_sm);
+
+// KV heads one decode CTA streams together (adjacent heads; only without GQA),
+// and query heads per decode unit (heads per CTA x KV heads per CTA).
+int32_t decode_kv_heads_per_cta(int32_t group, const pa_cache_desc& c);
+int32_t decode_heads_per_unit(int32_t group, const pa_cache_desc& c);
 // Heads of one GQA group handled together by one decode CTA.
 int32_t decode_heads_per_cta(int32_t group);
 // Decode smem stage geometry, used by the launcher and the API's checks.

@@ -394,16 +394,16 @@ cudaError_t launch_prefill_t(const PrefillArgs& a, const CUtensorMap& qmap, cons
   if (e != cudaSuccess) return e;
   if (dev < 64 && configured_smem[dev] < static_cast<int>(smem)) {
     e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
-    if (e != cudaSuccess) return e;
-    e = cudaFuncSetAttribute(kern, cudaFuncAttributePreferredSharedMemoryCarveout, cudaSharedmemCarveoutMaxShared);
-    if (e != cudaSuccess) return e;
+    if (e == cudaSuccess)
+      e = cudaFuncSetAttribute(kern, cudaFuncAttributePreferredSharedMemoryCarveout, cudaSharedmemCarveoutMaxShared);
+    if (e != cudaSuccess) {
+      (void)cudaGetLastError();  // reported through the return value; do not leave it pending
+      return e;
+    }
     configured_smem[dev] = static_cast<int>(smem);
   }
-  int per_sm = 0;
-  e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, 160, smem);
-  if (e != cudaSuccess) return e;
-  if (per_sm < 1) return cudaErrorInvalidConfiguration;
-  if (per_sm > 2) per_sm = 2;  // TMEM: 2 x 256 columns per SM
+  // TMEM holds 512 columns per SM; each CTA allocates kTmemCols of them.
+  const int per_sm = ctas_per_sm(reinterpret_cast<const void*>(kern), 160, smem, 512 / C::kTmemCols);
   const int64_t bound = static_cast<int64_t>(a.num_seqs) * (a.num_q_heads / GH) *
                         ((a.max_query_len + C::kTOK - 1) / C::kTOK);
   const int64_t slots = static_cast<int64_t>(num_sms()) * per_sm;
@@ -412,6 +412,7 @@ cudaError_t launch_prefill_t(const PrefillArgs& a, const CUtensorMap& qmap, cons
   // writes, so this grid may start as soon as SMs free up; each CTA waits for
   // the previous grid before it exits, which keeps stream order for whatever
   // is launched after pa_attention.
+  log_launch("paged_prefill_kernel", grid, 160, smem, per_sm);
   return launch_chained(kern, dim3(grid), dim3(160), smem, stream, qmap, kmap, vmap, a);
 }
 

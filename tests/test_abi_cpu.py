@@ -92,7 +92,7 @@ def test_attention_validation():
         _attn(num_q_heads=30)                                  # not a multiple of 8 kv heads
     assert e.value.status == P.PA_ERR_INVALID_ARG
     with pytest.raises(P.PAError) as e:
-        _attn()                                                # splits need a workspace
+        _attn()                                                # decode rows need a workspace
     assert e.value.status == P.PA_ERR_INVALID_ARG and "workspace" in str(e.value)
     need = P.pa_attention_workspace_size(4, 32, 1, 2048, DESC)
     with pytest.raises(P.PAError):
@@ -109,12 +109,14 @@ def test_attention_validation():
 
 
 def test_workspace_size_policy():
-    small = P.pa_attention_workspace_size(4, 32, 1, 32, DESC)
-    assert small == 0                                          # one split per sequence
-    big = P.pa_attention_workspace_size(32, 32, 1, 2048, (8192, 16, 32, 128, P.PA_BF16))
-    assert big > 0 and big % 4 == 0
+    a = P.pa_attention_workspace_size(4, 32, 1, 32, DESC)
+    b = P.pa_attention_workspace_size(4, 32, 1, 8192, DESC)
+    assert a == b > 0                                           # partial slots do not grow with context
+    big = P.pa_attention_workspace_size(64, 32, 1, 2048, DESC)
+    assert big > a and big % 4 == 0                            # they grow with sequences x heads
     assert P.pa_attention_workspace_size(4, 30, 1, 2048, DESC) == 0   # invalid -> 0
     assert P.pa_attention_workspace_size(4, 32, 0, 2048, DESC) == 0   # nothing to do
+    assert P.pa_attention_workspace_size(0, 32, 1, 2048, DESC) == 0
 
 
 # --------------------------------------------------------------------------

@@ -95,12 +95,30 @@ def test_random_decode_sweep(P, dtype, d, bs, g):
     _check_attention(got, o.out, dtype, "dtype=%s d=%d bs=%d g=%d" % (dtype, d, bs, g))
 
 
-@pytest.mark.parametrize("chunk", ["16", "64", "512"])
-def test_split_count_does_not_change_result(P, chunk, monkeypatch):
-    monkeypatch.setenv("PA_DECODE_CHUNK", chunk)
+@pytest.mark.parametrize("dtype", [W.BF16, W.FP32])
+@pytest.mark.parametrize("d", [64, 128])
+@pytest.mark.parametrize("bs", [8, 16, 32])
+def test_random_decode_multihead_sweep(P, dtype, d, bs):
+    """No GQA and a multiple of 4 KV heads: each CTA streams 4 adjacent heads."""
+    wl = _random_decode(3000 + d + bs, dtype, d, bs, 1, hkv=8)
+    b, o, got = _run_both(P, wl)
+    _check_attention(got, o.out, dtype, "multihead dtype=%s d=%d bs=%d" % (dtype, d, bs))
+
+
+@pytest.mark.parametrize("grid", ["1", "7", "64"])
+def test_grid_partition_does_not_change_result(P, grid, monkeypatch):
+    """Fewer decode CTAs move the partition boundaries (1 CTA: nothing is split)."""
+    monkeypatch.setenv("PA_DECODE_GRID", grid)
     wl = _random_decode(77, W.BF16, 128, 16, 4)
     b, o, got = _run_both(P, wl, check_caches=False)
-    _check_attention(got, o.out, W.BF16, "chunk " + chunk)
+    _check_attention(got, o.out, W.BF16, "grid " + grid)
+
+
+def test_single_long_sequence_split_over_many_ctas(P):
+    wl = W.random_case(78, num_seqs=1, q_lens=[1], ctx_extra=[8191], num_kv_heads=1, group=4, head_dim=128,
+                       block_size=16, dtype=W.BF16, max_blocks_per_seq=512)
+    b, o, got = _run_both(P, wl, check_caches=False)
+    _check_attention(got, o.out, W.BF16, "one sequence")
 
 
 def test_empty_and_zero_length_query_rows(P):
@@ -139,7 +157,9 @@ def test_out_of_range_indices_are_flagged_not_followed(P):
     tables = torch.tensor([[0, 77, -1, -1], [1, 2, 3, -1]], dtype=torch.int32, device=dev)
     lens = torch.tensor([20, 70], dtype=torch.int32, device=dev)       # seq 1 exceeds max_context_len
     qsl = torch.tensor([0, 1, 2], dtype=torch.int32, device=dev)
-    P.pa_attention(q, kc, vc, tables, 4, lens, qsl, 2, 2, 4, 1, 48, 0.125, desc, out, None, stream=None)
+    ws_bytes = P.pa_attention_workspace_size(2, 4, 1, 48, desc)
+    ws = torch.empty(ws_bytes, dtype=torch.uint8, device=dev)
+    P.pa_attention(q, kc, vc, tables, 4, lens, qsl, 2, 2, 4, 1, 48, 0.125, desc, out, ws, stream=None)
     flags = P.pa_read_device_flags(clear=True)
     assert flags & P.PA_FLAG_BLOCK_RANGE and flags & P.PA_FLAG_CONTEXT_RANGE
     assert not flags & P.PA_FLAG_WAIT_TIMEOUT
