@@ -353,8 +353,12 @@ def measure_kernels(b, reps: int = 10):
     row = geo.num_kv_heads * geo.head_dim * e
     res = {}
 
-    def timed(fn):
+    def timed(fn, tag):
         fn()
+        torch.cuda.synchronize(dev)
+        torch.cuda.nvtx.range_push(tag)  # lets a profiler select these calls
+        fn()
+        torch.cuda.nvtx.range_pop()
         torch.cuda.synchronize(dev)
         a, z = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         a.record()
@@ -371,7 +375,7 @@ def measure_kernels(b, reps: int = 10):
             if geo.dtype == "bf16" else torch.randn(n, geo.num_kv_heads, geo.head_dim, device=dev)
         sl = torch.from_numpy(slots).to(dev)
         kc2, vc2 = torch.empty_like(b.k_cache), torch.empty_like(b.v_cache)
-        ms = timed(lambda: P.pa_store_kv(kk, kk, sl, n, kc2, vc2, b.desc))
+        ms = timed(lambda: P.pa_store_kv(kk, kk, sl, n, kc2, vc2, b.desc), "pa_store_bulk")
         by = 4 * n * row + 4 * n
         res["store_bulk"] = {"tokens": n, "launch_ms": ms, "algorithmic_bytes": by, "gbs": by / (ms * 1e-3) / 1e9}
         del kk, kc2, vc2
@@ -381,7 +385,7 @@ def measure_kernels(b, reps: int = 10):
     npairs = min(len(free), len(used), 256)
     if npairs:
         pairs = torch.from_numpy(np.stack([used[:npairs], np.asarray(free[:npairs])], 1).astype(np.int32)).to(dev)
-        ms = timed(lambda: P.pa_copy_blocks(pairs, npairs, b.k_cache, b.v_cache, b.desc))
+        ms = timed(lambda: P.pa_copy_blocks(pairs, npairs, b.k_cache, b.v_cache, b.desc), "pa_copy")
         by = 4 * npairs * geo.block_size * row
         res["copy"] = {"pairs": npairs, "launch_ms": ms, "algorithmic_bytes": by, "gbs": by / (ms * 1e-3) / 1e9}
     pre = [i for i, q in enumerate(wl.q_lens) if q > 1]
@@ -397,7 +401,8 @@ def measure_kernels(b, reps: int = 10):
             torch.from_numpy(qsl).to(dev)
         out = torch.empty_like(b.out)
         ms = timed(lambda: P.pa_attention(b.q, b.k_cache, b.v_cache, bt, geo.max_blocks_per_seq, cl, qs, len(pre),
-                                          t, geo.num_q_heads, mq, ctx, wl.scale, b.desc, out, ws, ws_b))
+                                          t, geo.num_q_heads, mq, ctx, wl.scale, b.desc, out, ws, ws_b),
+                   "pa_prefill_only")
         flops = 0
         for i in pre:
             L, ql = int(lens[i]), wl.q_lens[i]
