@@ -156,3 +156,23 @@ def out_as_f64(t: torch.Tensor, dtype: str) -> np.ndarray:
 def cache_bits(t: torch.Tensor) -> np.ndarray:
     a = t.detach().cpu().numpy()
     return a.view(np.uint16) if a.dtype == np.int16 else a.view(np.uint32)
+
+
+def capture_step(b: DeviceBatch, pre=None, post=None):
+    """Capture one hot-path step (CoW copies, store, attention) in a CUDA graph.
+
+    ``pre`` / ``post`` are optional callables captured before / after the step
+    (e.g. host<->device copies of the step's inputs and output). Every libpa
+    call in the step is asynchronous, allocates nothing and never synchronises,
+    so the whole step can be replayed with one ``graph.replay()``. Run the step
+    once eagerly before capturing so one-time set-up (kernel attributes, the
+    tensor-map cache) happens outside the capture.
+    """
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g):
+        if pre is not None:
+            pre()
+        run_step(b)
+        if post is not None:
+            post()
+    return g
