@@ -248,6 +248,39 @@ int32_t pa_bm_seq_len(const pa_bm* bm, int64_t seq_id);
 /* Copy up to cap free-list entries (front first) to out; returns the count. */
 int32_t pa_bm_free_list(const pa_bm* bm, int32_t* out, int32_t cap);
 
+/*
+ * Block-manager statistics: the monitoring figures of [A] §"监控与调优要点"
+ * (block utilisation, target 70-85%; internal fragmentation, retune the block
+ * size above 20%; allocation latency P99, keep it under 1 ms; mapping-table
+ * memory, keep it under 1% of the KV cache) plus the saving from prefix
+ * sharing ([C] §"二、KV Cache管理：从浪费到极致复用").
+ */
+typedef struct {
+  int32_t num_blocks;             /* pool size */
+  int32_t free_blocks;            /* on the free list */
+  int32_t held_blocks;            /* refcount > 0 */
+  int32_t num_seqs;               /* live sequences */
+  int64_t logical_blocks;         /* table entries of all sequences (a shared block counts per holder) */
+  int64_t tokens;                 /* sum of sequence lengths */
+  int64_t used_slots;             /* slots of held blocks that hold a token (a shared slot counts once) */
+  double block_utilisation;       /* held_blocks / num_blocks */
+  double internal_fragmentation;  /* 1 - used_slots / (held_blocks * block_size) (0 if nothing held) */
+  double sharing_saving;          /* 1 - held_blocks / logical_blocks (0 if nothing held) */
+  double table_bytes;             /* 4 bytes (one int32 physical id) per table entry */
+  double table_overhead;          /* table_bytes / (num_blocks * kv_bytes_per_block): share of the whole KV pool */
+  double alloc_p50_us;            /* latency of block-allocating calls (add_seq, append_tokens) */
+  double alloc_p99_us;            /*   over the last (up to) 4096 such calls */
+  int64_t alloc_samples;
+} pa_bm_stats;
+
+/* Fill *out. kv_bytes_per_block: K+V bytes one physical block occupies across
+ * all layers (for table_overhead); pass 0 to leave table_overhead 0. A slot
+ * counts as used when some live sequence maps one of its tokens to it, so a
+ * shared block's used slots are those of the holder that wrote furthest.
+ * The latency window holds the last 4096 block-allocating calls; both
+ * percentiles are 0 before the first. Errors: PA_ERR_INVALID_ARG for NULL. */
+pa_status pa_bm_get_stats(const pa_bm* bm, double kv_bytes_per_block, pa_bm_stats* out);
+
 #ifdef __cplusplus
 }
 #endif

@@ -25,6 +25,7 @@ from .paged_kv import (  # noqa: F401
     kv_bytes_per_token,
     paged_attention,
     paged_attention_bruteforce,
+    preallocation_fragmentation,
     slot_of,
     store_kv,
     store_kv_bruteforce,

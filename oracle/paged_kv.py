@@ -400,3 +400,58 @@ class BlockManager:
             if self.ref[b] == 0:
                 self.free.append(b)
         del self.lens[seq_id]
+
+    # -- monitoring -------------------------------------------------------
+    def stats(self, kv_bytes_per_block: float = 0.0) -> dict:
+        """The pool's monitoring figures, from their definitions.
+
+        Source: [A] §"监控与调优要点": block utilisation is allocated blocks over
+        all blocks; internal fragmentation is the share of token slots inside
+        blocks that hold no token; the mapping-table memory is compared with the
+        whole KV cache. The saving from prefix sharing follows [C]
+        §"二、KV Cache管理：从浪费到极致复用" (several requests point at the same
+        pages).
+
+        Readings: a block is allocated while its reference count is positive; a
+        slot is used when some live sequence maps one of its tokens to it (the
+        set union over sequences, so a shared slot counts once); the mapping
+        table is one int32 physical id per logical block of every sequence; the
+        sharing saving is ``1 - physical / logical`` held blocks. Allocation
+        latency is a timing of the library's calls and has no oracle value.
+        """
+        held = [b for b in range(self.num_blocks) if self.ref[b] > 0]
+        used = set()
+        for sid, row in self.tables.items():
+            for p in range(self.lens[sid]):
+                used.add(slot_of(row, p, self.block_size))
+        logical = sum(len(row) for row in self.tables.values())
+        n_held = len(held)
+        table_bytes = 4.0 * logical
+        return dict(
+            num_blocks=self.num_blocks,
+            free_blocks=len(self.free),
+            held_blocks=n_held,
+            num_seqs=len(self.tables),
+            logical_blocks=logical,
+            tokens=sum(self.lens.values()),
+            used_slots=len(used),
+            block_utilisation=n_held / self.num_blocks if self.num_blocks else 0.0,
+            internal_fragmentation=1.0 - len(used) / (n_held * self.block_size) if n_held else 0.0,
+            sharing_saving=1.0 - n_held / logical if logical else 0.0,
+            table_bytes=table_bytes,
+            table_overhead=(table_bytes / (self.num_blocks * kv_bytes_per_block)
+                            if self.num_blocks and kv_bytes_per_block > 0 else 0.0),
+        )
+
+
+def preallocation_fragmentation(lengths, max_len: int) -> float:
+    """Unused share of a cache that reserves ``max_len`` token slots per request.
+
+    The contiguous scheme the pages compare against ([C] §"二、KV
+    Cache管理：从浪费到极致复用": allocate the maximum length up front): a
+    request of ``n`` tokens leaves ``max_len - n`` of its slots empty.
+    """
+    lengths = [int(n) for n in lengths]
+    if not lengths:
+        return 0.0
+    return 1.0 - sum(lengths) / (len(lengths) * max_len)

@@ -84,7 +84,21 @@ _SIGNATURES = {
     "pa_bm_refcount": (_I32, [_P, _I32]),
     "pa_bm_seq_len": (_I32, [_P, _I64]),
     "pa_bm_free_list": (_I32, [_P, _PI32, _I32]),
+    "pa_bm_get_stats": (C.c_int, [_P, C.c_double, C.c_void_p]),
 }
+
+
+class BlockManagerStats(C.Structure):
+    """Mirror of ``pa_bm_stats``."""
+    _fields_ = [("num_blocks", C.c_int32), ("free_blocks", C.c_int32), ("held_blocks", C.c_int32),
+                ("num_seqs", C.c_int32), ("logical_blocks", C.c_int64), ("tokens", C.c_int64),
+                ("used_slots", C.c_int64), ("block_utilisation", C.c_double),
+                ("internal_fragmentation", C.c_double), ("sharing_saving", C.c_double),
+                ("table_bytes", C.c_double), ("table_overhead", C.c_double), ("alloc_p50_us", C.c_double),
+                ("alloc_p99_us", C.c_double), ("alloc_samples", C.c_int64)]
+
+    def as_dict(self) -> dict:
+        return {name: getattr(self, name) for name, _ in self._fields_}
 
 _lib = None
 _lock = threading.Lock()
@@ -298,6 +312,12 @@ class BlockManager:
 
     def seq_len(self, seq_id: int) -> int:
         return int(self._lib.pa_bm_seq_len(self._h, int(seq_id)))
+
+    def stats(self, kv_bytes_per_block: float = 0.0) -> dict:
+        """``pa_bm_get_stats`` as a dict (monitoring figures of the pool)."""
+        st = BlockManagerStats()
+        _check(self._lib.pa_bm_get_stats(self._h, float(kv_bytes_per_block), C.byref(st)))
+        return st.as_dict()
 
     def free_list(self):
         n = self.num_blocks()

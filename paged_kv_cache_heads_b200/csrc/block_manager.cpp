@@ -17,6 +17,8 @@
 // more blocks than are free fails before changing anything; freed blocks
 // return in logical order; a write copies the shared last block only when
 // that block is partly filled (a full block is never written again).
+#include <algorithm>
+#include <chrono>
 #include <cstdint>
 #include <cstdio>
 #include <deque>
@@ -50,6 +52,22 @@ struct pa_bm {
   std::deque<int32_t> free_list;
   std::vector<int32_t> ref;
   std::unordered_map<int64_t, Sequence> seqs;
+  // latency of block-allocating calls, last kLatencyWindow samples (microseconds)
+  static constexpr size_t kLatencyWindow = 4096;
+  std::vector<float> latency_us;
+  size_t latency_next = 0;
+  int64_t latency_count = 0;
+
+  void record_latency(std::chrono::steady_clock::time_point t0) {
+    const float us = std::chrono::duration<float, std::micro>(std::chrono::steady_clock::now() - t0).count();
+    if (latency_us.size() < kLatencyWindow) {
+      latency_us.push_back(us);
+    } else {
+      latency_us[latency_next] = us;
+    }
+    latency_next = (latency_next + 1) % kLatencyWindow;
+    ++latency_count;
+  }
 
   int32_t take() {
     const int32_t b = free_list.front();
@@ -109,6 +127,7 @@ pa_status pa_bm_slot_mapping(const pa_bm* bm, int64_t seq_id, int32_t start, int
 
 pa_status pa_bm_add_seq(pa_bm* bm, int64_t seq_id, int32_t num_tokens, int32_t* slots_out) {
   if (!bm) return bm_fail(PA_ERR_INVALID_ARG, "bm is NULL");
+  const auto t0 = std::chrono::steady_clock::now();
   if (num_tokens < 0) return bm_fail(PA_ERR_INVALID_ARG, "num_tokens < 0");
   if (bm->seqs.count(seq_id)) return bm_fail(PA_ERR_INVALID_ARG, "sequence already exists");
   const int32_t need = blocks_for(num_tokens, bm->block_size);
@@ -119,6 +138,7 @@ pa_status pa_bm_add_seq(pa_bm* bm, int64_t seq_id, int32_t num_tokens, int32_t* 
   for (int32_t i = 0; i < need; ++i) seq.blocks.push_back(bm->take());
   seq.len = num_tokens;
   bm->seqs.emplace(seq_id, std::move(seq));
+  bm->record_latency(t0);
   if (slots_out) return pa_bm_slot_mapping(bm, seq_id, 0, num_tokens, slots_out);
   return PA_OK;
 }
@@ -145,6 +165,7 @@ pa_status pa_bm_append_tokens(pa_bm* bm, int64_t seq_id, int32_t n, int32_t* slo
   if (n < 0) return bm_fail(PA_ERR_INVALID_ARG, "n < 0");
   auto it = bm->seqs.find(seq_id);
   if (it == bm->seqs.end()) return bm_fail(PA_ERR_INDEX, "unknown sequence");
+  const auto t0 = std::chrono::steady_clock::now();
   Sequence& seq = it->second;
   const int32_t bs = bm->block_size;
   if (int64_t(seq.len) + n > INT32_MAX) return bm_fail(PA_ERR_INVALID_ARG, "sequence too long");
@@ -170,6 +191,7 @@ pa_status pa_bm_append_tokens(pa_bm* bm, int64_t seq_id, int32_t n, int32_t* slo
     if (slots_out) slots_out[i] = seq.blocks[p / bs] * bs + p % bs;
   }
   seq.len += n;
+  bm->record_latency(t0);
   return PA_OK;
 }
 
@@ -218,6 +240,48 @@ int32_t pa_bm_seq_len(const pa_bm* bm, int64_t seq_id) {
   if (!bm) return -1;
   auto it = bm->seqs.find(seq_id);
   return it == bm->seqs.end() ? -1 : it->second.len;
+}
+
+pa_status pa_bm_get_stats(const pa_bm* bm, double kv_bytes_per_block, pa_bm_stats* out) {
+  if (!bm || !out) return bm_fail(PA_ERR_INVALID_ARG, "NULL argument");
+  pa_bm_stats st = {};
+  const int32_t bs = bm->block_size;
+  st.num_blocks = bm->num_blocks;
+  st.free_blocks = static_cast<int32_t>(bm->free_list.size());
+  st.num_seqs = static_cast<int32_t>(bm->seqs.size());
+  // tokens a held block holds: the most any of its holders has written into it
+  std::vector<int32_t> fill(bm->num_blocks, 0);
+  for (const auto& kv : bm->seqs) {
+    const Sequence& seq = kv.second;
+    st.logical_blocks += static_cast<int64_t>(seq.blocks.size());
+    st.tokens += seq.len;
+    for (size_t i = 0; i < seq.blocks.size(); ++i) {
+      const int64_t in_block = std::min<int64_t>(bs, int64_t(seq.len) - int64_t(i) * bs);
+      fill[seq.blocks[i]] = std::max<int32_t>(fill[seq.blocks[i]], static_cast<int32_t>(in_block));
+    }
+  }
+  for (int32_t b = 0; b < bm->num_blocks; ++b)
+    if (bm->ref[b] > 0) {
+      ++st.held_blocks;
+      st.used_slots += fill[b];
+    }
+  st.block_utilisation = bm->num_blocks ? double(st.held_blocks) / bm->num_blocks : 0.0;
+  st.internal_fragmentation = st.held_blocks ? 1.0 - double(st.used_slots) / (double(st.held_blocks) * bs) : 0.0;
+  st.sharing_saving = st.logical_blocks ? 1.0 - double(st.held_blocks) / double(st.logical_blocks) : 0.0;
+  st.table_bytes = 4.0 * double(st.logical_blocks);
+  st.table_overhead = (bm->num_blocks && kv_bytes_per_block > 0)
+                          ? st.table_bytes / (double(bm->num_blocks) * kv_bytes_per_block)
+                          : 0.0;
+  if (!bm->latency_us.empty()) {
+    std::vector<float> v(bm->latency_us);
+    std::sort(v.begin(), v.end());
+    auto pct = [&](double q) { return double(v[std::min(v.size() - 1, size_t(q * (v.size() - 1) + 0.5))]); };
+    st.alloc_p50_us = pct(0.50);
+    st.alloc_p99_us = pct(0.99);
+  }
+  st.alloc_samples = bm->latency_count;
+  *out = st;
+  return PA_OK;
 }
 
 int32_t pa_bm_free_list(const pa_bm* bm, int32_t* out, int32_t cap) {

@@ -123,7 +123,18 @@ def test_workspace_size_policy():
 # libpa block manager == oracle block manager
 # --------------------------------------------------------------------------
 
+STAT_KEYS = ("num_blocks", "free_blocks", "held_blocks", "num_seqs", "logical_blocks", "tokens", "used_slots",
+             "block_utilisation", "internal_fragmentation", "sharing_saving", "table_bytes", "table_overhead")
+
+
+def _same_stats(a: P.BlockManager, b: oracle.BlockManager, kv_bytes_per_block=4096.0):
+    sa, sb = a.stats(kv_bytes_per_block), b.stats(kv_bytes_per_block)
+    for k in STAT_KEYS:
+        assert sa[k] == pytest.approx(sb[k], rel=1e-12, abs=1e-15), k
+
+
 def _same_state(a: P.BlockManager, b: oracle.BlockManager, live):
+    _same_stats(a, b)
     assert a.free_list() == list(b.free)
     assert [a.refcount(i) for i in range(b.num_blocks)] == list(b.ref)
     for s in live:
@@ -229,3 +240,29 @@ def test_block_manager_errors():
     with pytest.raises(P.PAError):
         P.BlockManager(3, 16, [0, 0, 1])                       # not a permutation
     assert bm.refcount(99) == -1 and bm.seq_len(42) == -1
+
+
+def test_block_manager_allocation_latency_window():
+    """Allocation latency: one sample per successful add/append; P99 under the
+    1 ms bound of [A] §"监控与调优要点" for a pool of the decode batch's size."""
+    wl = W.llama7b_decode()
+    geo = wl.geometry
+    a = P.BlockManager(geo.num_blocks, geo.block_size, wl.initial_free_order)
+    st = a.stats()
+    assert st["alloc_samples"] == 0 and st["alloc_p99_us"] == 0.0
+    calls = 0
+    for op in wl.ops:
+        if op.kind == "add":
+            a.add_seq(op.seq, op.n)
+            calls += 1
+        elif op.kind == "append":
+            a.append_tokens(op.seq, op.n)
+            calls += 1
+    for i in range(5000):                                   # more calls than the window
+        a.append_tokens(wl.batch_seqs[i % len(wl.batch_seqs)], 1)
+    with pytest.raises(P.PAError):
+        a.add_seq(10 ** 9, geo.num_blocks * geo.block_size)  # a failed call is not a sample
+    st = a.stats()
+    assert st["alloc_samples"] == calls + 5000
+    assert 0.0 < st["alloc_p50_us"] <= st["alloc_p99_us"] < 1000.0
+    assert st["table_overhead"] == 0.0                      # no per-block size given
