@@ -275,6 +275,10 @@ def measure_ours(wl, steps: int, warmup: int, device, gpu_index: int):
     P.load_library()
     P.pa_read_device_flags(clear=True)
     b = gs.prepare(wl, device)
+    geo = wl.geometry
+    # K+V bytes of one block of this single-layer cache: the table's share is that of one layer
+    per_block = 2 * geo.block_size * geo.num_kv_heads * geo.head_dim * (2 if geo.dtype == "bf16" else 4)
+    bm_stats = b.host["bm"].stats(per_block)
     stream = torch.cuda.current_stream(device)
     for _ in range(max(warmup, 1)):
         gs.run_step(b)
@@ -370,7 +374,7 @@ def measure_ours(wl, steps: int, warmup: int, device, gpu_index: int):
     del graph
     kernels = measure_kernels(b)
     flags = P.pa_read_device_flags(clear=True)
-    return dict(kernels=kernels, step_mode="cuda_graph" if ms_graph <= ms_eager else "eager",
+    return dict(bm_stats=bm_stats, kernels=kernels, step_mode="cuda_graph" if ms_graph <= ms_eager else "eager",
                 step_eager_ms=ms_eager / steps, step_graph_ms=ms_graph / steps, e2e_eager_ms=e2e_eager_ms, e2e_graph_ms=e2e_graph_ms, ms_total=ms_total, attn_ms=attn_ms, e2e_ms=e2e_ms, h2d=h2d, d2h=d2h, clocks=clocks.summary(),
                 launches=launches_per_step(b) * steps, step_tokens=b.num_step_tokens,
                 step_pairs=int(b.step_pairs.shape[0]), flags=flags, max_context_len=b.max_context_len)
@@ -564,6 +568,7 @@ def main():
                             "graph_ms_per_step": r["step_graph_ms"]},
             "gpu_launches": r["launches"], "clocks": r["clocks"], "device_flags": r["flags"],
             "kernels": kern,
+            "block_manager": {k: (round(v, 6) if isinstance(v, float) else v) for k, v in r["bm_stats"].items()},
             "step_bytes": work["attn_bytes"] + work["store_bytes"] + work["copy_bytes"]}
     print(json.dumps(line), flush=True)
     return 0

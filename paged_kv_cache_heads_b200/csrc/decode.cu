@@ -37,42 +37,12 @@
 //    kernel merges them: O = sum_c 2^(lse_c - M) O_c / sum_c 2^(lse_c - M).
 #include <math_constants.h>
 
+#include "decode_common.cuh"
 #include "pa_common.cuh"
 #include "pa_internal.h"
 
 namespace pa {
 namespace {
-
-// First CTA whose range [c*B/G, (c+1)*B/G) contains block b (0 <= b < B).
-__device__ __forceinline__ int cta_of_block(int64_t b, int64_t B, int G) {
-  return static_cast<int>(((b + 1) * G - 1) / B);
-}
-
-// Block-wide inclusive scan of one int per thread (nthreads <= 1024).
-__device__ __forceinline__ int block_inclusive_scan(int x, int* warp_tot, int& total) {
-  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, nw = (blockDim.x + 31) >> 5;
-#pragma unroll
-  for (int off = 1; off < 32; off <<= 1) {
-    const int y = __shfl_up_sync(0xffffffffu, x, off);
-    if (lane >= off) x += y;
-  }
-  if (lane == 31) warp_tot[warp] = x;
-  __syncthreads();
-  if (warp == 0) {
-    int t = lane < nw ? warp_tot[lane] : 0;
-#pragma unroll
-    for (int off = 1; off < 32; off <<= 1) {
-      const int y = __shfl_up_sync(0xffffffffu, t, off);
-      if (lane >= off) t += y;
-    }
-    if (lane < nw) warp_tot[lane] = t;
-  }
-  __syncthreads();
-  total = warp_tot[nw - 1];
-  const int r = x + (warp > 0 ? warp_tot[warp - 1] : 0);
-  __syncthreads();
-  return r;
-}
 
 // KH > 1 (only with GH == 1, KH == NCW): the CTA streams KH adjacent KV heads
 // at once -- one TMA box {D, KH, bs, 1} reads KH*D contiguous elements per
@@ -117,15 +87,6 @@ struct DecodeCfg {
   static_assert(KH == 1 || (GH == 1 && KH == NCW), "multi-head CTAs: one warp per KV head");
   static_assert(kLogGH <= kLogLPR, "more heads than lanes per row");
   static size_t smem_bytes(int num_seqs) { return 1024 + kSeqOff + 12ull * (num_seqs + 1); }
-};
-
-// One segment: the part of a unit's block range that one CTA streams.
-struct Segment {
-  int s;         // sequence
-  int hg;        // head group (first query head hg * GH)
-  int blo, bhi;  // logical blocks [blo, bhi) of the sequence
-  int L;         // context length
-  int slot;      // partial slot (unit + cta), or -1 when this CTA covers the whole unit
 };
 
 template <typename T, int D, int BS, int GH, int KH, int NCW>
@@ -192,6 +153,10 @@ __global__ void __launch_bounds__((NCW + 1) * 32, (GH == 1 ? 4 : 3))
     carry += total;
   }
   __syncthreads();
+  // Chained launch: everything above overlaps the previous grid; the cache
+  // (written by a preceding store) and the workspace (read by a preceding
+  // merge) are touched only after it has completed.
+  grid_dependency_wait();
   const int64_t B = static_cast<int64_t>(prefix[a.num_seqs]) * HG;  // blocks of all units
   if (blockIdx.x == 0 && a.seq_prefix)
     for (int i = tid; i <= a.num_seqs; i += blockDim.x) a.seq_prefix[i] = prefix[i];
@@ -200,22 +165,8 @@ __global__ void __launch_bounds__((NCW + 1) * 32, (GH == 1 ? 4 : 3))
 
   // the segment of this CTA that starts at global block b (beg <= b < end)
   auto segment_at = [&](int64_t b, Segment& g) {
-    int lo = 0, hi = a.num_seqs;  // largest s with prefix[s] * HG <= b
-    while (hi - lo > 1) {
-      const int mid = (lo + hi) >> 1;
-      if (static_cast<int64_t>(prefix[mid]) * HG <= b) lo = mid; else hi = mid;
-    }
-    const int nbs = prefix[lo + 1] - prefix[lo];
-    const int64_t off = b - static_cast<int64_t>(prefix[lo]) * HG;
-    const int hg = static_cast<int>(off / nbs);
-    const int lb = static_cast<int>(off - static_cast<int64_t>(hg) * nbs);
-    const int64_t ub0 = b - lb, ub1 = ub0 + nbs;  // the unit's global block range
-    g.s = lo;
-    g.hg = hg;
-    g.blo = lb;
-    g.bhi = lb + static_cast<int>(min(static_cast<int64_t>(nbs - lb), end - b));
-    g.L = clen[lo];
-    g.slot = (ub0 >= beg && ub1 <= end) ? -1 : (lo * HG + hg) + static_cast<int>(blockIdx.x);
+    locate_segment(b, prefix, a.num_seqs, HG, beg, end, static_cast<int>(blockIdx.x), g);
+    g.L = clen[g.s];
   };
 
   if (warp == NCW) {
@@ -591,8 +542,7 @@ cudaError_t launch_decode_t(DecodeArgs& a, const CUtensorMap& kmap, const CUtens
   }
   a.grid = grid;
   log_launch("paged_decode_kernel", grid, C::kThreads, smem, per_sm);
-  kern<<<grid, C::kThreads, smem, stream>>>(kmap, vmap, a);
-  return cudaGetLastError();
+  return launch_chained(kern, dim3(grid), dim3(C::kThreads), smem, stream, kmap, vmap, a);
 }
 
 template <typename T, int D, int BS>
@@ -628,6 +578,7 @@ cudaError_t launch_combine_t(const DecodeArgs& a, cudaStream_t stream) {
 template <typename T, int D, int BS>
 cudaError_t launch_combine_gh(const DecodeArgs& a, const pa_cache_desc& desc, cudaStream_t stream) {
   switch (decode_heads_per_unit(a.num_q_heads / a.num_kv_heads, desc)) {
+    case 8: return launch_combine_t<T, D, BS, 8>(a, stream);
     case 4: return launch_combine_t<T, D, BS, 4>(a, stream);
     case 2: return launch_combine_t<T, D, BS, 2>(a, stream);
     default: return launch_combine_t<T, D, BS, 1>(a, stream);
@@ -659,6 +610,7 @@ int32_t decode_kv_heads_per_cta(int32_t group, const pa_cache_desc& c) {
 }
 
 int32_t decode_heads_per_unit(int32_t group, const pa_cache_desc& c) {
+  if (decode_uses_tc(group, c)) return group;  // one unit per KV head
   return decode_heads_per_cta(group) * decode_kv_heads_per_cta(group, c);
 }
 

@@ -368,11 +368,25 @@ pa_status pa_attention(const void* q, const void* k_cache, const void* v_cache,
   a.grid = 0;
   a.scale_log2 = scale_log2;
 
+  const int32_t group = num_q_heads / cache->num_kv_heads;
+  // q as a 3-D tensor {head_dim, num_q_heads, num_q_tokens} (decode and prefill maps)
+  const uint64_t qd[3] = {uint64_t(cache->head_dim), uint64_t(num_q_heads), uint64_t(num_q_tokens)};
+  const uint64_t qs[2] = {uint64_t(cache->head_dim) * 2, uint64_t(num_q_heads) * cache->head_dim * 2};
   CUtensorMap kmap, vmap;
-  const uint32_t kh = decode_kv_heads_per_cta(num_q_heads / cache->num_kv_heads, *cache);
-  if ((st = cache_map(&kmap, k_cache, *cache, cache->head_dim, 0, kh)) != PA_OK) return st;
-  if ((st = cache_map(&vmap, v_cache, *cache, cache->head_dim, 0, kh)) != PA_OK) return st;
-  e = launch_decode(a, kmap, vmap, *cache, s);
+  if (decode_uses_tc(group, *cache)) {
+    // tensor-core decode: 64-column (128-byte) swizzled boxes, Q^T per KV head
+    CUtensorMap qmap;
+    const uint32_t qbox[3] = {64, uint32_t(group), 1};
+    if ((st = tensor_map(&qmap, q, 3, qd, qs, qbox, PA_BF16, 128)) != PA_OK) return st;
+    if ((st = cache_map(&kmap, k_cache, *cache, 64, 128)) != PA_OK) return st;
+    if ((st = cache_map(&vmap, v_cache, *cache, 64, 128)) != PA_OK) return st;
+    e = launch_decode_tc(a, qmap, kmap, vmap, *cache, s);
+  } else {
+    const uint32_t kh = decode_kv_heads_per_cta(group, *cache);
+    if ((st = cache_map(&kmap, k_cache, *cache, cache->head_dim, 0, kh)) != PA_OK) return st;
+    if ((st = cache_map(&vmap, v_cache, *cache, cache->head_dim, 0, kh)) != PA_OK) return st;
+    e = launch_decode(a, kmap, vmap, *cache, s);
+  }
   if (e != cudaSuccess) return cuda_fail(e, "decode launch");
   e = launch_decode_combine(a, *cache, s);
   if (e != cudaSuccess) return cuda_fail(e, "decode combine launch");
@@ -392,12 +406,9 @@ pa_status pa_attention(const void* q, const void* k_cache, const void* v_cache,
     p.max_query_len = max_query_len;
     p.num_q_tokens = num_q_tokens;
     p.scale_log2 = scale_log2;
-    // Q as a 3-D tensor {head_dim, num_q_heads, num_q_tokens}; K/V boxes are
-    // 64 columns wide (128 bytes) to match the 128-byte swizzle of the MMA tiles.
-    const uint64_t qd[3] = {uint64_t(cache->head_dim), uint64_t(num_q_heads), uint64_t(num_q_tokens)};
-    const uint64_t qs[2] = {uint64_t(cache->head_dim) * 2, uint64_t(num_q_heads) * cache->head_dim * 2};
-    const int32_t g = num_q_heads / cache->num_kv_heads;
-    const int32_t gh = prefill_heads_per_tile(g);
+    // K/V boxes are 64 columns wide (128 bytes) to match the 128-byte swizzle
+    // of the MMA tiles.
+    const int32_t gh = prefill_heads_per_tile(group);
     const uint32_t qbox[3] = {64, uint32_t(gh), uint32_t(128 / gh)};
     CUtensorMap qmap, pk, pv;
     if ((st = tensor_map(&qmap, q, 3, qd, qs, qbox, PA_BF16, 128)) != PA_OK) return st;

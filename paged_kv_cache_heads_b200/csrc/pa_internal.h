@@ -66,6 +66,13 @@ cudaError_t launch_copy_blocks(const int32_t* pairs, int32_t num_pairs, void* k_
                                cudaStream_t stream);
 cudaError_t launch_decode(DecodeArgs& a, const CUtensorMap& kmap, const CUtensorMap& vmap,
                           const pa_cache_desc& c, cudaStream_t stream);
+// Grouped-query decode on the tensor cores: bf16, head_dim 128, group 2, 4 or 8
+// (environment PA_DECODE_TC=0 selects the CUDA-core kernel instead). `qmap` is
+// q as {head_dim, num_q_heads, num_q_tokens} with box {64, group, 1}; the cache
+// maps have box {64, 1, block_size, 1}; all three use the 128-byte swizzle.
+bool decode_uses_tc(int32_t group, const pa_cache_desc& c);
+cudaError_t launch_decode_tc(DecodeArgs& a, const CUtensorMap& qmap, const CUtensorMap& kmap,
+                             const CUtensorMap& vmap, const pa_cache_desc& c, cudaStream_t stream);
 cudaError_t launch_decode_combine(const DecodeArgs& a, const pa_cache_desc& c, cudaStream_t stream);
 cudaError_t launch_prefill(const PrefillArgs& a, const CUtensorMap& qmap, const CUtensorMap& kmap,
                            const CUtensorMap& vmap, const pa_cache_desc& c, cudaStream_t stream);

@@ -34,6 +34,9 @@ __global__ void __launch_bounds__(kThreads) store_kv_kernel(
     const uint4* __restrict__ k, const uint4* __restrict__ v, const int32_t* __restrict__ slots,
     uint32_t num_tokens, uint32_t n16, uint32_t num_slots, uint4* __restrict__ k_cache,
     uint4* __restrict__ v_cache, unsigned* status) {
+  // A chained attention grid may start its prologue now; it waits for this
+  // grid's completion before it reads the cache.
+  launch_dependents();
   const uint32_t per_tensor = num_tokens * n16;
   const uint32_t total = 2u * per_tensor;
   const uint32_t stride = gridDim.x * blockDim.x;
@@ -73,6 +76,7 @@ __global__ void __launch_bounds__(kThreads) copy_blocks_kernel(const int32_t* __
                                                               uint4* __restrict__ k_cache,
                                                               uint4* __restrict__ v_cache,
                                                               uint32_t chunks, unsigned* status) {
+  launch_dependents();
   const uint32_t pair = blockIdx.x;
   const uint32_t tensor = blockIdx.y / chunks;
   const uint32_t chunk = blockIdx.y - tensor * chunks;

@@ -239,3 +239,68 @@ def test_prefill_large_logits_trigger_rescale(P):
             op.k = W.f32_to_bf16_bits(f * ramp)
     b, o, got = _run_both(P, wl)
     _check_attention(got, o.out, W.BF16, "rescale")
+
+
+# --------------------------------------------------------------------------
+# grouped-query decode on the tensor cores (bf16, head_dim 128, group 2/4/8)
+# --------------------------------------------------------------------------
+
+def test_decode_large_logits_trigger_rescale(P):
+    """Keys scaled up along each sequence so the running max keeps growing:
+    exercises the lazy rescale of l and of the O^T columns between tiles."""
+    wl = _random_decode(4242, W.BF16, 128, 16, 4, hkv=2)
+    for op in wl.ops:
+        if op.k is not None and op.k.size:
+            f = W.bf16_bits_to_f32(op.k)
+            ramp = np.linspace(0.5, 8.0, f.shape[0], dtype=np.float32)[:, None, None]
+            op.k = W.f32_to_bf16_bits(f * ramp)
+    b, o, got = _run_both(P, wl)
+    _check_attention(got, o.out, W.BF16, "decode rescale")
+
+
+def test_decode_many_sequences_two_stage_ring(P):
+    """4600 short sequences: the per-sequence table in shared memory leaves room
+    for only two 64 KiB stages, which selects the two-stage variant."""
+    rng = np.random.default_rng(4600)
+    n = 4600
+    lens = rng.integers(1, 48, size=n)
+    wl = W.random_case(4600, num_seqs=n, q_lens=[1] * n, ctx_extra=[int(x) - 1 for x in lens], num_kv_heads=1,
+                       group=8, head_dim=128, block_size=16, dtype=W.BF16)
+    b, o, got = _run_both(P, wl, check_caches=False)
+    _check_attention(got, o.out, W.BF16, "many sequences")
+
+
+_CUDA_CORE_SCRIPT = r'''
+import sys, numpy as np, torch
+sys.path.insert(0, sys.argv[1])
+from oracle import scenario as oscen
+from paged_kv_cache_heads_b200 import workloads as W, scenario as gs
+import paged_kv_cache_heads_b200 as P
+worst = 0.0
+for seed, g, bs in [(11, 4, 16), (12, 2, 8), (13, 8, 32)]:
+    rng = np.random.default_rng(seed)
+    lens = [1, bs + 1, int(rng.integers(600, 1400)), int(rng.integers(2000, 2600))]
+    wl = W.random_case(seed, num_seqs=4, q_lens=[1] * 4, ctx_extra=[x - 1 for x in lens], num_kv_heads=2,
+                       group=g, head_dim=128, block_size=bs, dtype=W.BF16)
+    b = gs.prepare(wl)
+    gs.run_step(b)
+    torch.cuda.synchronize()
+    o = oscen.run(wl, W.sentinel_cache(wl.geometry), W.sentinel_cache(wl.geometry))
+    err = np.abs(gs.out_as_f64(b.out, W.BF16) - o.out)
+    assert np.isfinite(err).all() and err.max() <= 2e-2 and err.mean() <= 2e-3, (seed, err.max(), err.mean())
+    worst = max(worst, float(err.max()))
+assert P.pa_read_device_flags(clear=True) == 0
+print("OK", worst)
+'''
+
+
+def test_cuda_core_grouped_decode_still_matches(P):
+    """PA_DECODE_TC=0 keeps the CUDA-core grouped kernel reachable; it must
+    stay within tolerance too (it serves fp32 and head_dim 64)."""
+    import subprocess
+    import sys
+    root = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+    env = dict(os.environ, PA_DECODE_TC="0")
+    r = subprocess.run([sys.executable, "-c", _CUDA_CORE_SCRIPT, root], capture_output=True, text=True, env=env,
+                       cwd=root, timeout=600)
+    assert r.returncode == 0 and "OK" in r.stdout, r.stdout + r.stderr
