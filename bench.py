@@ -386,7 +386,10 @@ def measure_kernels(b, reps: int = 10):
     * store_bulk: one pa_store_kv of every cached token of the batch (their
       slots, fresh rows) -- the bandwidth-bound bulk fill;
     * copy: pa_copy_blocks of 256 block pairs (src = a used block, dst = a free one);
-    * prefill_only: pa_attention over the sequences with q_len > 1 alone.
+    * prefill_only: pa_attention over the sequences with q_len > 1 alone;
+    * compaction: the block manager's remap of the held blocks into a dense
+      range, and the pa_copy_blocks call that moves their data (last: it
+      rewrites the host tables, so nothing runs on this batch afterwards).
     Each is timed with CUDA events over ``reps`` back-to-back calls after a warm-up.
     """
     import torch
@@ -454,6 +457,19 @@ def measure_kernels(b, reps: int = 10):
             flops += 4 * geo.head_dim * geo.num_q_heads * sum(L - ql + j + 1 for j in range(ql))
         res["prefill_only"] = {"seqs": len(pre), "q_tokens": t, "launch_ms": ms, "flops": flops,
                                "tflops": flops / (ms * 1e-3) / 1e12}
+    # compaction: the block manager remaps every held block into [0, held) and
+    # pa_copy_blocks moves their K/V data (repeating the copy is idempotent)
+    bm = b.host["bm"]
+    held_blocks = bm.num_blocks() - bm.num_free()
+    t0 = time.perf_counter()
+    moves = bm.compact()
+    host_ms = (time.perf_counter() - t0) * 1e3
+    if moves:
+        dp = torch.tensor(moves, dtype=torch.int32, device=dev)
+        ms = timed(lambda: P.pa_copy_blocks(dp, len(moves), b.k_cache, b.v_cache, b.desc), "pa_compact_copy")
+        by = 4 * len(moves) * geo.block_size * row
+        res["compaction"] = {"moves": len(moves), "held_blocks": held_blocks, "host_remap_ms": host_ms,
+                             "launch_ms": ms, "algorithmic_bytes": by, "gbs": by / (ms * 1e-3) / 1e9}
     return res
 
 
@@ -546,7 +562,7 @@ def main():
             "algorithmic_bytes_per_launch": work["attn_bytes"], "launch_ms": attn_ms,
             "kv_read_gbs": work["attn_kv_bytes"] / (attn_ms * 1e-3) / 1e9}
     kern = r["kernels"]
-    for k in ("store_bulk", "copy"):
+    for k in ("store_bulk", "copy", "compaction"):
         if k in kern:
             kern[k]["frac_of_hbm_peak"] = kern[k]["gbs"] / hbm_peak
     if "prefill_only" in kern:

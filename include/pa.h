@@ -249,6 +249,24 @@ int32_t pa_bm_seq_len(const pa_bm* bm, int64_t seq_id);
 int32_t pa_bm_free_list(const pa_bm* bm, int32_t* out, int32_t cap);
 
 /*
+ * Compaction ([A] §"连续批处理与内存管理的协同": defragmentation remaps blocks so
+ * the used memory becomes dense, at the price of moving data). Every held
+ * block ends in the id range [0, H), H = number of held blocks: the held
+ * blocks with id >= H, in ascending order, move to the free ids below H, in
+ * ascending order. Every table entry and reference count moves with its
+ * block; the free list becomes H, H+1, ..., num_blocks-1.
+ *
+ * Writes the moves as (src, dst) int32 pairs to pairs_out (host memory, room
+ * for `cap` pairs) and their count to *num_pairs_out. The caller copies the
+ * K/V data with pa_copy_blocks(pairs, n, ...) before any attention that
+ * reads the new tables (sources and destinations are disjoint, so one call in
+ * any order suffices); n is the migration cost in blocks.
+ * Errors: PA_ERR_INVALID_ARG for NULL arguments or when cap < n, in which case
+ * *num_pairs_out is still set to n and nothing changes.
+ */
+pa_status pa_bm_compact(pa_bm* bm, int32_t* pairs_out, int32_t cap, int32_t* num_pairs_out);
+
+/*
  * Block-manager statistics: the monitoring figures of [A] §"监控与调优要点"
  * (block utilisation, target 70-85%; internal fragmentation, retune the block
  * size above 20%; allocation latency P99, keep it under 1 ms; mapping-table

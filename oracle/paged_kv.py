@@ -401,6 +401,30 @@ class BlockManager:
                 self.free.append(b)
         del self.lens[seq_id]
 
+    def compact(self) -> list[tuple[int, int]]:
+        """Remap every held block into the dense id range ``[0, H)``.
+
+        Source: [A] §"连续批处理与内存管理的协同" lists defragmentation by block
+        remapping ("memory compaction") and warns that moving blocks costs
+        bandwidth. Readings: H is the number of held blocks; the held blocks
+        whose id is H or more, taken in ascending order, move to the free ids
+        below H, taken in ascending order; tables and reference counts follow
+        their blocks; afterwards the free list is H, H+1, ..., num_blocks-1.
+        Returns the ``(src, dst)`` moves; their count is the migration cost.
+        """
+        held = [b for b in range(self.num_blocks) if self.ref[b] > 0]
+        h = len(held)
+        movers = [b for b in held if b >= h]
+        holes = [b for b in range(h) if self.ref[b] == 0]
+        assert len(movers) == len(holes)
+        remap = dict(zip(movers, holes))
+        for src, dst in remap.items():
+            self.ref[dst], self.ref[src] = self.ref[src], 0
+        for sid in self.tables:
+            self.tables[sid] = [remap.get(b, b) for b in self.tables[sid]]
+        self.free = deque(range(h, self.num_blocks))
+        return list(zip(movers, holes))
+
     # -- monitoring -------------------------------------------------------
     def stats(self, kv_bytes_per_block: float = 0.0) -> dict:
         """The pool's monitoring figures, from their definitions.

@@ -85,6 +85,7 @@ _SIGNATURES = {
     "pa_bm_seq_len": (_I32, [_P, _I64]),
     "pa_bm_free_list": (_I32, [_P, _PI32, _I32]),
     "pa_bm_get_stats": (C.c_int, [_P, C.c_double, C.c_void_p]),
+    "pa_bm_compact": (C.c_int, [_P, _PI32, _I32, _PI32]),
 }
 
 
@@ -312,6 +313,18 @@ class BlockManager:
 
     def seq_len(self, seq_id: int) -> int:
         return int(self._lib.pa_bm_seq_len(self._h, int(seq_id)))
+
+    def compact(self):
+        """``pa_bm_compact``: remap held blocks to [0, held); returns the (src, dst) moves."""
+        import numpy as np
+        n = C.c_int32(0)
+        status = self._lib.pa_bm_compact(self._h, None, 0, C.byref(n))  # size query; no moves -> done
+        if n.value == 0:
+            _check(status)
+            return []
+        pairs = np.empty((n.value, 2), dtype=np.int32)
+        _check(self._lib.pa_bm_compact(self._h, pairs.ctypes.data_as(_PI32), n.value, C.byref(n)))
+        return [(int(a), int(b)) for a, b in pairs]
 
     def stats(self, kv_bytes_per_block: float = 0.0) -> dict:
         """``pa_bm_get_stats`` as a dict (monitoring figures of the pool)."""

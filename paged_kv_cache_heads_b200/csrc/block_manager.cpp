@@ -242,6 +242,39 @@ int32_t pa_bm_seq_len(const pa_bm* bm, int64_t seq_id) {
   return it == bm->seqs.end() ? -1 : it->second.len;
 }
 
+pa_status pa_bm_compact(pa_bm* bm, int32_t* pairs_out, int32_t cap, int32_t* num_pairs_out) {
+  if (!bm || !num_pairs_out) return bm_fail(PA_ERR_INVALID_ARG, "NULL argument");
+  if (cap < 0) return bm_fail(PA_ERR_INVALID_ARG, "negative capacity");
+  int32_t held = 0;
+  for (int32_t b = 0; b < bm->num_blocks; ++b) held += bm->ref[b] > 0;
+  // movers: held blocks at or past `held`; holes: free ids below it (both ascending)
+  std::vector<int32_t> map(bm->num_blocks);
+  for (int32_t b = 0; b < bm->num_blocks; ++b) map[b] = b;
+  int32_t n = 0, hole = 0;
+  for (int32_t b = held; b < bm->num_blocks; ++b) {
+    if (bm->ref[b] == 0) continue;
+    while (bm->ref[hole] > 0) ++hole;  // a hole exists below `held` for every mover
+    map[b] = hole++;
+    ++n;
+  }
+  *num_pairs_out = n;
+  if (n > cap || (n > 0 && !pairs_out)) return bm_fail(PA_ERR_INVALID_ARG, "pairs_out holds fewer than the moves");
+  int32_t k = 0;
+  for (int32_t b = held; b < bm->num_blocks; ++b) {
+    if (map[b] == b) continue;
+    pairs_out[2 * k] = b;
+    pairs_out[2 * k + 1] = map[b];
+    ++k;
+    bm->ref[map[b]] = bm->ref[b];
+    bm->ref[b] = 0;
+  }
+  for (auto& kv : bm->seqs)
+    for (int32_t& b : kv.second.blocks) b = map[b];
+  bm->free_list.clear();
+  for (int32_t b = held; b < bm->num_blocks; ++b) bm->free_list.push_back(b);
+  return PA_OK;
+}
+
 pa_status pa_bm_get_stats(const pa_bm* bm, double kv_bytes_per_block, pa_bm_stats* out) {
   if (!bm || !out) return bm_fail(PA_ERR_INVALID_ARG, "NULL argument");
   pa_bm_stats st = {};

@@ -195,11 +195,13 @@ def test_block_manager_matches_oracle_on_random_ops(seed):
                 assert ra == "oob"
             else:
                 assert ra[0] == rb[0] and [tuple(p) for p in ra[1]] == [tuple(p) for p in rb[1]]
-        else:
+        elif r < 0.97:
             s = int(rng.choice(live))
             a.free_seq(s)
             b.free_seq(s)
             live.remove(s)
+        else:
+            assert a.compact() == b.compact()
         _same_state(a, b, live)
     for s in live:
         assert a.slot_mapping(s, 0, b.seq_len(s)) == b.slot_mapping(s, 0, b.seq_len(s))
@@ -266,3 +268,28 @@ def test_block_manager_allocation_latency_window():
     assert st["alloc_samples"] == calls + 5000
     assert 0.0 < st["alloc_p50_us"] <= st["alloc_p99_us"] < 1000.0
     assert st["table_overhead"] == 0.0                      # no per-block size given
+
+
+def test_compaction_matches_oracle_on_workloads():
+    for name in ("prefix_cow", "mixed_bs8"):
+        wl = W.CONFIGS[name]()
+        geo = wl.geometry
+        a = P.BlockManager(geo.num_blocks, geo.block_size, wl.initial_free_order)
+        b = oracle.BlockManager(geo.num_blocks, geo.block_size, wl.initial_free_order)
+        for op in wl.ops:
+            if op.kind == "add":
+                a.add_seq(op.seq, op.n)
+                b.add_seq(op.seq, op.n)
+            elif op.kind == "fork":
+                a.fork(op.parent, op.seq, op.n)
+                b.fork(op.parent, op.seq, op.n)
+            elif op.kind == "append":
+                a.append_tokens(op.seq, op.n)
+                b.append_tokens(op.seq, op.n)
+        for s in wl.batch_seqs[::3]:
+            a.free_seq(s)
+            b.free_seq(s)
+        live = [s for s in wl.batch_seqs if s not in wl.batch_seqs[::3]]
+        pa_, pb = a.compact(), b.compact()
+        assert pa_ == pb and len(pa_) > 0
+        _same_state(a, b, live)

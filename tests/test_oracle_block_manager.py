@@ -303,3 +303,55 @@ def test_stats_count_planted_double_counting():
     bm.fork(0, 1)
     per_holder = sum(bm.seq_len(s) for s in bm.tables)
     assert per_holder == 12 and bm.stats()["used_slots"] == 6
+
+
+# --------------------------------------------------------------------------
+# compaction ([A] §"连续批处理与内存管理的协同": remap blocks, weigh the moves)
+# --------------------------------------------------------------------------
+
+def _scattered_pool(seed, nb=64, bs=4):
+    rng = np.random.default_rng(seed)
+    bm = BlockManager(nb, bs, rng.permutation(nb))
+    for s in range(12):
+        bm.add_seq(s, int(rng.integers(0, 5 * bs)))
+    bm.fork(3, 100)
+    bm.fork(5, 101, max(0, bm.seq_len(5) - 3))
+    bm.append_tokens(101, 2)
+    for s in (0, 4, 7, 9):
+        bm.free_seq(s)
+    return bm
+
+
+@pytest.mark.parametrize("seed", range(6))
+def test_compaction_makes_held_blocks_dense_and_keeps_every_token(seed):
+    bm = _scattered_pool(seed)
+    bs = bm.block_size
+    # give every slot a value that names (block, row), then move the data as the pairs say
+    cache = np.arange(bm.num_blocks * bs, dtype=np.int64).reshape(bm.num_blocks, bs)
+    before = {s: [cache[b, p % bs] for p in range(bm.seq_len(s)) for b in [bm.blocks_of(s)[p // bs]]]
+              for s in bm.tables}
+    refs_before = sorted(bm.ref[b] for b in range(bm.num_blocks) if bm.ref[b] > 0)
+    held = sum(1 for b in range(bm.num_blocks) if bm.ref[b] > 0)
+    pairs = bm.compact()
+    for src, dst in pairs:
+        assert src >= held > dst                        # moves only from above the dense range into it
+        cache[dst] = cache[src]
+    assert len({d for _, d in pairs}) == len(pairs) == len({s for s, _ in pairs})
+    assert {b for b in range(bm.num_blocks) if bm.ref[b] > 0} == set(range(held))
+    assert list(bm.free) == list(range(held, bm.num_blocks))
+    assert sorted(bm.ref[b] for b in range(held)) == refs_before
+    after = {s: [cache[b, p % bs] for p in range(bm.seq_len(s)) for b in [bm.blocks_of(s)[p // bs]]]
+             for s in bm.tables}
+    assert after == before
+    check_invariants(bm)
+    assert bm.compact() == []                           # already dense: nothing moves
+
+
+def test_compaction_order_is_ascending_movers_to_ascending_holes():
+    bm = BlockManager(8, 2, [7, 5, 3, 0, 1, 2, 4, 6])
+    bm.add_seq(0, 4)                                    # blocks 7, 5
+    bm.add_seq(1, 2)                                    # block 3
+    # H = 3 held blocks, all at ids >= 3: 3 -> 0, 5 -> 1, 7 -> 2
+    assert bm.compact() == [(3, 0), (5, 1), (7, 2)]
+    assert bm.blocks_of(0) == [2, 1] and bm.blocks_of(1) == [0]
+    assert list(bm.free) == [3, 4, 5, 6, 7]
