@@ -387,6 +387,8 @@ def measure_kernels(b, reps: int = 10):
       slots, fresh rows) -- the bandwidth-bound bulk fill;
     * copy: pa_copy_blocks of 256 block pairs (src = a used block, dst = a free one);
     * prefill_only: pa_attention over the sequences with q_len > 1 alone;
+    * cascade: pa_attention_cascade on the batch when its sequences share
+      leading blocks (bytes actually read: each group's shared blocks once);
     * compaction: the block manager's remap of the held blocks into a dense
       range, and the pa_copy_blocks call that moves their data (last: it
       rewrites the host tables, so nothing runs on this batch afterwards).
@@ -457,6 +459,24 @@ def measure_kernels(b, reps: int = 10):
             flops += 4 * geo.head_dim * geo.num_q_heads * sum(L - ql + j + 1 for j in range(ql))
         res["prefill_only"] = {"seqs": len(pre), "q_tokens": t, "launch_ms": ms, "flops": flops,
                                "tflops": flops / (ms * 1e-3) / 1e12}
+    # cascade: when sequences of the batch share leading blocks, the same
+    # attention with each group's shared blocks read once
+    plan = gs.plan_cascade(b) if all(q == 1 for q in wl.q_lens) else None
+    if plan is not None and plan.num_groups:
+        out = torch.empty_like(b.out)
+        ms = timed(lambda: gs.run_attention_cascade(b, plan, out=out), "pa_cascade")
+        shared, groups = plan.host["shared"], plan.host["groups"]
+        lens = b.host["context_lens"]
+        tok_bytes = 2 * geo.num_kv_heads * geo.head_dim * e
+        # keys each sequence reads itself, plus each group's shared blocks once
+        own = sum(int(L) - int(sh) * geo.block_size for L, sh in zip(lens, shared))
+        once = sum(int(shared[f]) * geo.block_size for f, _ in groups)
+        unique = (own + once) * tok_bytes
+        logical = int(np.sum(lens)) * tok_bytes
+        res["cascade"] = {"groups": int(len(groups)), "shared_blocks": int(plan.max_shared_blocks),
+                          "members": int(sum(int(c) for _, c in groups)), "launch_ms": ms,
+                          "kv_bytes_read": unique, "kv_bytes_logical": logical,
+                          "gbs": unique / (ms * 1e-3) / 1e9, "logical_gbs": logical / (ms * 1e-3) / 1e9}
     # compaction: the block manager remaps every held block into [0, held) and
     # pa_copy_blocks moves their K/V data (repeating the copy is idempotent)
     bm = b.host["bm"]
@@ -562,7 +582,7 @@ def main():
             "algorithmic_bytes_per_launch": work["attn_bytes"], "launch_ms": attn_ms,
             "kv_read_gbs": work["attn_kv_bytes"] / (attn_ms * 1e-3) / 1e9}
     kern = r["kernels"]
-    for k in ("store_bulk", "copy", "compaction"):
+    for k in ("store_bulk", "copy", "compaction", "cascade"):
         if k in kern:
             kern[k]["frac_of_hbm_peak"] = kern[k]["gbs"] / hbm_peak
     if "prefill_only" in kern:

@@ -175,6 +175,41 @@ pa_status pa_attention_static_workspace(const void* q, const void* k_cache, cons
                                         const pa_cache_desc* cache, void* out, void* stream);
 
 /*
+ * pa_attention_cascade -- decode attention that reads shared prefix blocks
+ * once per group ("vLLM核心架构：PagedAttention原理、KV Cache管理、连续批处理机制",
+ * §"二、KV Cache管理：从浪费到极致复用": requests with a common prefix point at
+ * the same pages; here the shared pages are also read only once).
+ *
+ * Same result as pa_attention for a batch of decode rows (every sequence has
+ * exactly one query row: query_start_loc[s] = s, q is [num_seqs, Hq, D]):
+ * out[s, h] = softmax(q[s, h] . K_s[0:L_s]^T * scale) . V_s[0:L_s].
+ * Group g is the groups[2g+1] >= 2 consecutive sequences starting at
+ * groups[2g] (groups are disjoint); every member s of a group has shared_blocks[s] = n_g,
+ * the same n_g >= 1 leading block-table entries as the group's first member,
+ * all of them full (n_g * block_size <= L_s). shared_blocks[s] = 0 for a
+ * sequence in no group. The n_g shared blocks are attended once for all
+ * members (a tensor-core pass over their stacked query rows, in chunks of 256
+ * tokens); each member streams only its own blocks past them; the two partial
+ * results are merged with their log-sum-exp weights.
+ *   shared_blocks  device [num_seqs] int32     groups  device [num_groups][2] int32 (first, count)
+ *   max_group_size >= the largest group; max_shared_blocks >= every n_g
+ *                  (<= max_blocks_per_seq); both bound the launch and the workspace
+ *   workspace      >= pa_attention_cascade_workspace_size(...) bytes, 16-byte aligned
+ * bf16 caches only (PA_ERR_UNSUPPORTED otherwise). Other arguments, errors and
+ * device flags as pa_attention; a group that breaks the rules above raises
+ * PA_FLAG_CONTEXT_RANGE and its members' rows are unspecified.
+ */
+size_t pa_attention_cascade_workspace_size(int32_t num_seqs, int32_t num_q_heads, int32_t max_context_len,
+                                           int32_t max_shared_blocks, const pa_cache_desc* cache);
+pa_status pa_attention_cascade(const void* q, const void* k_cache, const void* v_cache,
+                               const int32_t* block_tables, int32_t max_blocks_per_seq,
+                               const int32_t* context_lens, const int32_t* query_start_loc, int32_t num_seqs,
+                               int32_t num_q_heads, int32_t max_context_len, const int32_t* shared_blocks,
+                               const int32_t* groups, int32_t num_groups, int32_t max_group_size,
+                               int32_t max_shared_blocks, float scale, const pa_cache_desc* cache, void* out,
+                               void* workspace, size_t workspace_bytes, void* stream);
+
+/*
  * pa_read_device_flags -- read (and optionally clear) the device status word
  * of the current device. Synchronises the device first (all streams).
  *   flags  host out: OR of PA_FLAG_* raised since the last clear
@@ -247,6 +282,19 @@ int32_t pa_bm_refcount(const pa_bm* bm, int32_t block);
 int32_t pa_bm_seq_len(const pa_bm* bm, int64_t seq_id);
 /* Copy up to cap free-list entries (front first) to out; returns the count. */
 int32_t pa_bm_free_list(const pa_bm* bm, int32_t* out, int32_t cap);
+
+/*
+ * Groups for pa_attention_cascade, from the block tables of seq_ids (host, n
+ * sequences, in batch order). Consecutive sequences form a group while the
+ * number of leading block-table entries they all share, counting only blocks
+ * full in every member, stays >= min_shared_blocks (>= 1); a group needs two
+ * members or more. Writes shared_out[n] (that count for members, 0 for the
+ * rest), groups_out (room for n/2 (first, count) pairs) and *num_groups_out.
+ * Errors: PA_ERR_INVALID_ARG (NULL, n < 0, min_shared_blocks < 1), PA_ERR_INDEX
+ * (unknown sequence).
+ */
+pa_status pa_bm_cascade_groups(const pa_bm* bm, const int64_t* seq_ids, int32_t n, int32_t min_shared_blocks,
+                               int32_t* shared_out, int32_t* groups_out, int32_t* num_groups_out);
 
 /*
  * Compaction ([A] §"连续批处理与内存管理的协同": defragmentation remaps blocks so

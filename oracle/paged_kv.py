@@ -425,6 +425,47 @@ class BlockManager:
         self.free = deque(range(h, self.num_blocks))
         return list(zip(movers, holes))
 
+    def cascade_groups(self, seq_ids, min_shared_blocks: int = 1):
+        """Runs of consecutive sequences that share leading full blocks.
+
+        Source: [C] §"二、KV Cache管理：从浪费到极致复用" (requests with a common
+        prefix point at the same pages, so those pages can be read once for
+        all of them). Readings: a group is a run of at least two consecutive
+        sequences of the batch; its shared count is the number of leading
+        block-table entries identical in every member and full in every member
+        (index < length // block_size); runs are taken greedily from the left,
+        each as long as its shared count stays >= min_shared_blocks.
+        Returns (shared [n] with each member's count and 0 elsewhere,
+        groups [(first, count), ...]).
+        """
+        ids = list(seq_ids)
+        n = len(ids)
+        rows = [self.tables[s] for s in ids]
+        full = [self.lens[s] // self.block_size for s in ids]
+
+        def shared_count(i, j):  # members i .. j-1
+            k = 0
+            while all(k < full[m] for m in range(i, j)) and all(rows[m][k] == rows[i][k] for m in range(i, j)):
+                k += 1
+            return k
+
+        shared = [0] * n
+        groups = []
+        i = 0
+        while i < n:
+            j = i + 1
+            while j < n and shared_count(i, j + 1) >= min_shared_blocks:
+                j += 1
+            if j - i >= 2:
+                c = shared_count(i, j)
+                groups.append((i, j - i))
+                for m in range(i, j):
+                    shared[m] = c
+                i = j
+            else:
+                i += 1
+        return shared, groups
+
     # -- monitoring -------------------------------------------------------
     def stats(self, kv_bytes_per_block: float = 0.0) -> dict:
         """The pool's monitoring figures, from their definitions.

@@ -86,6 +86,10 @@ _SIGNATURES = {
     "pa_bm_free_list": (_I32, [_P, _PI32, _I32]),
     "pa_bm_get_stats": (C.c_int, [_P, C.c_double, C.c_void_p]),
     "pa_bm_compact": (C.c_int, [_P, _PI32, _I32, _PI32]),
+    "pa_bm_cascade_groups": (C.c_int, [_P, _PI64, _I32, _I32, _PI32, _PI32, _PI32]),
+    "pa_attention_cascade_workspace_size": (C.c_size_t, [_I32, _I32, _I32, _I32, C.POINTER(CacheDesc)]),
+    "pa_attention_cascade": (C.c_int, [_P, _P, _P, _P, _I32, _P, _P, _I32, _I32, _I32, _P, _P, _I32, _I32, _I32,
+                                       C.c_float, C.POINTER(CacheDesc), _P, _P, C.c_size_t, _P]),
 }
 
 
@@ -222,6 +226,28 @@ def pa_attention_static_workspace(q, k_cache, v_cache, block_tables, max_blocks_
         _stream(stream, q, out)))
 
 
+def pa_attention_cascade_workspace_size(num_seqs, num_q_heads, max_context_len, max_shared_blocks, cache) -> int:
+    d = _desc(cache)
+    return int(load_library().pa_attention_cascade_workspace_size(int(num_seqs), int(num_q_heads),
+                                                                  int(max_context_len), int(max_shared_blocks),
+                                                                  C.byref(d)))
+
+
+def pa_attention_cascade(q, k_cache, v_cache, block_tables, max_blocks_per_seq, context_lens, query_start_loc,
+                         num_seqs, num_q_heads, max_context_len, shared_blocks, groups, num_groups, max_group_size,
+                         max_shared_blocks, scale, cache, out, workspace, workspace_bytes=None, stream=None):
+    """Decode attention reading each group's shared prefix blocks once (see include/pa.h)."""
+    d = _desc(cache)
+    if workspace_bytes is None:
+        workspace_bytes = 0 if workspace is None or isinstance(workspace, int) else \
+            workspace.numel() * workspace.element_size()
+    _check(load_library().pa_attention_cascade(
+        _ptr(q), _ptr(k_cache), _ptr(v_cache), _ptr(block_tables), int(max_blocks_per_seq), _ptr(context_lens),
+        _ptr(query_start_loc), int(num_seqs), int(num_q_heads), int(max_context_len), _ptr(shared_blocks),
+        _ptr(groups), int(num_groups), int(max_group_size), int(max_shared_blocks), float(scale), C.byref(d),
+        _ptr(out), _ptr(workspace), int(workspace_bytes), _stream(stream, q, out)))
+
+
 def pa_read_device_flags(clear: bool = True) -> int:
     """OR of PA_FLAG_* raised on the current device since the last clear (synchronises)."""
     v = C.c_uint32(0)
@@ -325,6 +351,19 @@ class BlockManager:
         pairs = np.empty((n.value, 2), dtype=np.int32)
         _check(self._lib.pa_bm_compact(self._h, pairs.ctypes.data_as(_PI32), n.value, C.byref(n)))
         return [(int(a), int(b)) for a, b in pairs]
+
+    def cascade_groups(self, seq_ids, min_shared_blocks: int = 1):
+        """``pa_bm_cascade_groups``: (shared_blocks [n] int32, groups [g, 2] int32) for pa_attention_cascade."""
+        import numpy as np
+        ids = np.ascontiguousarray(seq_ids, dtype=np.int64)
+        n = len(ids)
+        shared = np.zeros(max(n, 1), dtype=np.int32)
+        groups = np.zeros((max(n // 2, 1), 2), dtype=np.int32)
+        ng = C.c_int32(0)
+        _check(self._lib.pa_bm_cascade_groups(self._h, ids.ctypes.data_as(_PI64), n, int(min_shared_blocks),
+                                              shared.ctypes.data_as(_PI32), groups.ctypes.data_as(_PI32),
+                                              C.byref(ng)))
+        return shared[:n], groups[: ng.value]
 
     def stats(self, kv_bytes_per_block: float = 0.0) -> dict:
         """``pa_bm_get_stats`` as a dict (monitoring figures of the pool)."""

@@ -242,6 +242,44 @@ int32_t pa_bm_seq_len(const pa_bm* bm, int64_t seq_id) {
   return it == bm->seqs.end() ? -1 : it->second.len;
 }
 
+pa_status pa_bm_cascade_groups(const pa_bm* bm, const int64_t* seq_ids, int32_t n, int32_t min_shared_blocks,
+                               int32_t* shared_out, int32_t* groups_out, int32_t* num_groups_out) {
+  if (!bm || n < 0 || min_shared_blocks < 1 || !num_groups_out || (n > 0 && (!seq_ids || !shared_out || !groups_out)))
+    return bm_fail(PA_ERR_INVALID_ARG, "bad cascade_groups arguments");
+  std::vector<const Sequence*> seq(n);
+  for (int32_t i = 0; i < n; ++i) {
+    auto it = bm->seqs.find(seq_ids[i]);
+    if (it == bm->seqs.end()) return bm_fail(PA_ERR_INDEX, "unknown sequence");
+    seq[i] = &it->second;
+    shared_out[i] = 0;
+  }
+  auto full_blocks = [&](int32_t i) { return seq[i]->len / bm->block_size; };
+  int32_t groups = 0, i = 0;
+  while (i < n) {
+    // extend [i, j) while the members still share >= min_shared_blocks full leading blocks
+    int32_t common = full_blocks(i), j = i + 1;
+    while (j < n) {
+      const int32_t c = std::min(common, full_blocks(j));
+      int32_t k = 0;
+      while (k < c && seq[j]->blocks[k] == seq[i]->blocks[k]) ++k;
+      if (k < min_shared_blocks) break;
+      common = k;
+      ++j;
+    }
+    if (j - i >= 2 && common >= min_shared_blocks) {
+      groups_out[2 * groups] = i;
+      groups_out[2 * groups + 1] = j - i;
+      ++groups;
+      for (int32_t m = i; m < j; ++m) shared_out[m] = common;
+      i = j;
+    } else {
+      ++i;
+    }
+  }
+  *num_groups_out = groups;
+  return PA_OK;
+}
+
 pa_status pa_bm_compact(pa_bm* bm, int32_t* pairs_out, int32_t cap, int32_t* num_pairs_out) {
   if (!bm || !num_pairs_out) return bm_fail(PA_ERR_INVALID_ARG, "NULL argument");
   if (cap < 0) return bm_fail(PA_ERR_INVALID_ARG, "negative capacity");

@@ -123,9 +123,6 @@ __global__ void __launch_bounds__((NCW + 1) * 32, (GH == 1 ? 4 : 3))
     tma_prefetch_desc(&kmap);
     tma_prefetch_desc(&vmap);
   }
-  // The merge kernel (and any prefill grid) may be scheduled now; the merge
-  // waits for this grid's completion before it reads a partial.
-  launch_dependents();
 
   // ---- decode blocks of every sequence, and their prefix
   int carry = 0;
@@ -140,10 +137,12 @@ __global__ void __launch_bounds__((NCW + 1) * 32, (GH == 1 ? 4 : 3))
       clen[s] = L;
       qrow[s] = r0;
       if (ql == 1) {
-        if (L < 1 || L > a.max_context_len || L > a.max_blocks_per_seq * BS) {
+        const int skip = a.skip_blocks ? __ldg(a.skip_blocks + s) : 0;
+        if (L < 1 || L > a.max_context_len || L > a.max_blocks_per_seq * BS || skip < 0 ||
+            skip > (L + BS - 1) / BS) {
           raise_flag(a.status, PA_FLAG_CONTEXT_RANGE);
         } else {
-          n = (L + BS - 1) / BS;
+          n = (L + BS - 1) / BS - skip;
         }
       }
     }
@@ -155,8 +154,11 @@ __global__ void __launch_bounds__((NCW + 1) * 32, (GH == 1 ? 4 : 3))
   __syncthreads();
   // Chained launch: everything above overlaps the previous grid; the cache
   // (written by a preceding store) and the workspace (read by a preceding
-  // merge) are touched only after it has completed.
+  // merge) are touched only after it has completed. Only then may the grids
+  // chained after this one start: they read the same cache, and each of them
+  // waits for its own predecessor at most.
   grid_dependency_wait();
+  launch_dependents();
   const int64_t B = static_cast<int64_t>(prefix[a.num_seqs]) * HG;  // blocks of all units
   if (blockIdx.x == 0 && a.seq_prefix)
     for (int i = tid; i <= a.num_seqs; i += blockDim.x) a.seq_prefix[i] = prefix[i];
@@ -166,6 +168,7 @@ __global__ void __launch_bounds__((NCW + 1) * 32, (GH == 1 ? 4 : 3))
   // the segment of this CTA that starts at global block b (beg <= b < end)
   auto segment_at = [&](int64_t b, Segment& g) {
     locate_segment(b, prefix, a.num_seqs, HG, beg, end, static_cast<int>(blockIdx.x), g);
+    apply_skip(a.skip_blocks, HG, static_cast<int>(blockIdx.x), g);
     g.L = clen[g.s];
   };
 
@@ -175,7 +178,7 @@ __global__ void __launch_bounds__((NCW + 1) * 32, (GH == 1 ? 4 : 3))
     // segment's loads are issued, so a segment never waits on a table read.
     auto fetch_ids = [&](const Segment& g, int b0) {  // raw ids; checked when used
       return b0 + lane < g.bhi
-                 ? __ldg(a.block_tables + static_cast<size_t>(g.s) * a.max_blocks_per_seq + b0 + lane)
+                 ? __ldg(a.block_tables + static_cast<size_t>(g.s) * a.max_blocks_per_seq + g.skip + b0 + lane)
                  : 0;
     };
     auto checked = [&](int phys) {
@@ -272,7 +275,7 @@ __global__ void __launch_bounds__((NCW + 1) * 32, (GH == 1 ? 4 : 3))
       if (!mbar_wait(&full[st], (kk / C::kNST) & 1, a.status)) { ok = false; break; }
       const uint8_t* Ks = smem + st * C::kStageB + (KH > 1 ? warp * C::kRowB : 0);
       const uint8_t* Vs = Ks + BS * C::kTokB;
-      const int tok0 = (blo + i) * BS;
+      const int tok0 = (g.skip + blo + i) * BS;
 #pragma unroll
       for (int u = 0; u < C::kNUPD; ++u) {
         float sc[C::kNIT];
@@ -439,9 +442,10 @@ __global__ void __launch_bounds__((NCW + 1) * 32, (GH == 1 ? 4 : 3))
 }
 
 // One CTA per unit (sequence, head group), GH x D threads: merge the
-// partials of a unit that several CTAs streamed. The weights
-// 2^(lse_c - M) / sum are formed in parallel in shared memory, then each
-// thread sums its (head, column) over the covering CTAs.
+// partials of a unit that several CTAs streamed and, for a cascade sequence,
+// the prefix-pass partials of its shared blocks. The weights
+// 2^(lse_j - M) / sum are formed in parallel in shared memory, then each
+// thread sums its (head, column) over the partials.
 template <typename T, int D, int BS, int GH>  // GH here: query heads per unit
 __global__ void __launch_bounds__(GH * D) decode_combine_kernel(const DecodeArgs a) {
   launch_dependents();
@@ -451,24 +455,36 @@ __global__ void __launch_bounds__(GH * D) decode_combine_kernel(const DecodeArgs
   const int u = blockIdx.x;
   const int s = u / HG, hg = u - s * HG;
   const int nbs = a.seq_prefix[s + 1] - a.seq_prefix[s];
-  if (nbs == 0) return;
-  const int64_t B = static_cast<int64_t>(a.seq_prefix[a.num_seqs]) * HG;
-  const int64_t ub0 = static_cast<int64_t>(a.seq_prefix[s]) * HG + static_cast<int64_t>(hg) * nbs;
-  const int c0 = cta_of_block(ub0, B, a.grid);
-  const int c1 = cta_of_block(ub0 + nbs - 1, B, a.grid);
-  if (c0 == c1) return;  // one CTA covered the unit and wrote its rows
-  const int n = c1 - c0 + 1;
+  const int skip = a.skip_blocks ? __ldg(a.skip_blocks + s) : 0;
+  const int n1 = skip > 0 ? (skip + a.l1_chunk_blocks - 1) / a.l1_chunk_blocks : 0;  // prefix-pass chunks
+  if (nbs == 0 && n1 == 0) return;
+  int c0 = 0, n2 = 0;  // covering decode CTAs c0 .. c0 + n2 - 1
+  if (nbs > 0) {
+    const int64_t B = static_cast<int64_t>(a.seq_prefix[a.num_seqs]) * HG;
+    const int64_t ub0 = static_cast<int64_t>(a.seq_prefix[s]) * HG + static_cast<int64_t>(hg) * nbs;
+    c0 = cta_of_block(ub0, B, a.grid);
+    n2 = cta_of_block(ub0 + nbs - 1, B, a.grid) - c0 + 1;
+    if (n2 == 1 && n1 == 0) return;  // one CTA covered the unit and wrote its rows
+  }
+  const int n = n2 + n1;
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   float* mx = wsm + n * GH;
   float* sm = mx + GH;
   const size_t slot0 = static_cast<size_t>(u) + c0;
-  // With more CTAs than blocks some CTAs in [c0, c1] stream nothing and wrote
-  // no partial: they get weight 0 (and their slot is never read).
+  const size_t l1_row = static_cast<size_t>(s) * a.num_q_heads + static_cast<size_t>(hg) * GH;  // + gi
+  // With more CTAs than blocks some CTAs in [c0, c0 + n2) stream nothing and
+  // wrote no partial: they get weight 0 (and their slot is never read).
   auto streams = [&](int cc) {
-    return static_cast<int64_t>(cc) * B / a.grid < static_cast<int64_t>(cc + 1) * B / a.grid;
+    return static_cast<int64_t>(cc) * (static_cast<int64_t>(a.seq_prefix[a.num_seqs]) * HG) / a.grid <
+           static_cast<int64_t>(cc + 1) * (static_cast<int64_t>(a.seq_prefix[a.num_seqs]) * HG) / a.grid;
   };
-  for (int i = tid; i < n * GH; i += blockDim.x)
-    wsm[i] = streams(c0 + i / GH) ? a.part_lse[slot0 * GH + i] : -CUDART_INF_F;
+  for (int i = tid; i < n * GH; i += blockDim.x) {
+    const int j = i / GH, gi = i - j * GH;
+    if (j < n2)
+      wsm[i] = streams(c0 + j) ? a.part_lse[(slot0 + j) * GH + gi] : -CUDART_INF_F;
+    else
+      wsm[i] = a.l1_lse[(l1_row + gi) * a.l1_max_chunks + (j - n2)];
+  }
   __syncthreads();
   if (warp < GH) {  // warp g reduces head g over the n partials
     float m = -CUDART_INF_F;
@@ -492,12 +508,14 @@ __global__ void __launch_bounds__(GH * D) decode_combine_kernel(const DecodeArgs
   __syncthreads();
   const int gi = tid / D, d = tid - gi * D;
   const float* po = a.part_o + (slot0 * GH + gi) * D + d;
+  const float* p1 = a.l1_o + ((l1_row + gi) * a.l1_max_chunks) * D + d;
   const size_t stride = static_cast<size_t>(GH) * D;
   float o0 = 0.f, o1 = 0.f, o2 = 0.f, o3 = 0.f;
   int j = 0;
   auto term = [&](int jj) {  // weight 0 marks a CTA without a partial: skip its stale slot
     const float w = wsm[jj * GH + gi];
-    return w != 0.f ? w * po[jj * stride] : 0.f;
+    if (w == 0.f) return 0.f;
+    return w * (jj < n2 ? po[jj * stride] : p1[static_cast<size_t>(jj - n2) * D]);
   };
   for (; j + 4 <= n; j += 4) {
     o0 += term(j);
@@ -570,7 +588,7 @@ cudaError_t launch_decode_bs(DecodeArgs& a, const CUtensorMap& kmap, const CUten
 template <typename T, int D, int BS, int GH>
 cudaError_t launch_combine_t(const DecodeArgs& a, cudaStream_t stream) {
   auto kern = decode_combine_kernel<T, D, BS, GH>;
-  const size_t smem = (static_cast<size_t>(a.grid) + 2) * GH * sizeof(float);
+  const size_t smem = (static_cast<size_t>(a.grid) + a.l1_max_chunks + 2) * GH * sizeof(float);
   const unsigned grid = static_cast<unsigned>(a.num_seqs) * (a.num_q_heads / GH);
   return launch_chained(kern, dim3(grid), dim3(GH * D), smem, stream, a);
 }

@@ -52,6 +52,7 @@ struct Segment {
   int blo, bhi;  // logical blocks [blo, bhi) of the sequence
   int L;         // context length (filled by the caller)
   int slot;      // partial slot (unit + cta), or -1 when this CTA covers the whole unit
+  int skip;      // leading table blocks left to the cascade prefix pass (0 without cascade)
 };
 
 // The segment of CTA `cta`, whose range is [beg, end), that starts at global
@@ -74,6 +75,15 @@ __device__ __forceinline__ void locate_segment(int64_t b, const int* prefix, int
   g.blo = lb;
   g.bhi = lb + static_cast<int>(nbs - lb < end - b ? nbs - lb : end - b);
   g.slot = (ub0 >= beg && ub1 <= end) ? -1 : (lo * HG + hg) + cta;
+  g.skip = 0;
+}
+
+// Cascade decode: a sequence whose first `skip` blocks the prefix pass reads
+// streams only blocks [skip, ...) and always leaves a partial for the merge.
+__device__ __forceinline__ void apply_skip(const int32_t* skip_blocks, int HG, int cta, Segment& g) {
+  if (!skip_blocks) return;
+  g.skip = __ldg(skip_blocks + g.s);
+  if (g.skip > 0 && g.slot < 0) g.slot = (g.s * HG + g.hg) + cta;
 }
 
 }  // namespace pa

@@ -87,6 +87,7 @@ struct DecTcCfg {
 template <int kBlk>
 struct TileWalk {
   const int* prefix;
+  const int32_t* skip_blocks;
   int num_seqs, HG, cta;
   int64_t beg, end, next_b;
   Segment g;
@@ -94,8 +95,10 @@ struct TileWalk {
   int seg;        // segment counter (from 0)
   bool valid;
 
-  __device__ __forceinline__ void start(const int* p, int S, int hg, int64_t b0, int64_t b1, int c) {
+  __device__ __forceinline__ void start(const int* p, const int32_t* skip, int S, int hg, int64_t b0, int64_t b1,
+                                        int c) {
     prefix = p;
+    skip_blocks = skip;
     num_seqs = S;
     HG = hg;
     beg = b0;
@@ -109,6 +112,7 @@ struct TileWalk {
     valid = next_b < end;
     if (!valid) return;
     locate_segment(next_b, prefix, num_seqs, HG, beg, end, cta, g);
+    apply_skip(skip_blocks, HG, cta, g);
     next_b += g.bhi - g.blo;
     tb = g.blo;
     ++seg;
@@ -170,8 +174,6 @@ __global__ void __launch_bounds__(192, 1)
     tma_prefetch_desc(&kmap);
     tma_prefetch_desc(&vmap);
   }
-  // The merge kernel may be scheduled now; it waits for this grid to complete.
-  launch_dependents();
 
   // ---- decode blocks of every sequence, and their prefix
   int carry = 0;
@@ -184,10 +186,12 @@ __global__ void __launch_bounds__(192, 1)
       const int r0 = __ldg(a.query_start_loc + s);
       const int ql = __ldg(a.query_start_loc + s + 1) - r0;
       if (ql == 1) {
-        if (L < 1 || L > a.max_context_len || L > a.max_blocks_per_seq * BS) {
+        const int skip = a.skip_blocks ? __ldg(a.skip_blocks + s) : 0;
+        if (L < 1 || L > a.max_context_len || L > a.max_blocks_per_seq * BS || skip < 0 ||
+            skip > (L + BS - 1) / BS) {
           raise_flag(a.status, PA_FLAG_CONTEXT_RANGE);
         } else {
-          n = (L + BS - 1) / BS;
+          n = (L + BS - 1) / BS - skip;
         }
       }
     }
@@ -201,8 +205,11 @@ __global__ void __launch_bounds__(192, 1)
   tc::fence_after_sync();
   // Chained launch: everything above overlaps the previous grid; the cache
   // (written by a preceding store) and the workspace (read by a preceding
-  // merge) are touched only after it has completed.
+  // merge) are touched only after it has completed. Only then may the grids
+  // chained after this one start: they read the same cache, and each of them
+  // waits for its own predecessor at most.
   grid_dependency_wait();
+  launch_dependents();
   const uint32_t tmem = *tmem_slot;
   const int64_t B = static_cast<int64_t>(prefix[a.num_seqs]) * HG;  // blocks of all units
   if (blockIdx.x == 0 && a.seq_prefix)
@@ -211,7 +218,7 @@ __global__ void __launch_bounds__(192, 1)
   const int64_t end = static_cast<int64_t>(blockIdx.x + 1) * B / a.grid;
 
   TileWalk<C::kBlk> it;
-  it.start(prefix, a.num_seqs, HG, beg, end, static_cast<int>(blockIdx.x));
+  it.start(prefix, a.skip_blocks, a.num_seqs, HG, beg, end, static_cast<int>(blockIdx.x));
 
   if (warp == 4) {
     // ================= producer: Q^T per segment, K and V per block (TMA)
@@ -240,7 +247,7 @@ __global__ void __launch_bounds__(192, 1)
       // block index -1, an out-of-range box that TMA fills with zeros
       int phys = -1;
       if (lane < it.blocks()) {
-        phys = __ldg(a.block_tables + static_cast<size_t>(g.s) * a.max_blocks_per_seq + it.tb + lane);
+        phys = __ldg(a.block_tables + static_cast<size_t>(g.s) * a.max_blocks_per_seq + g.skip + it.tb + lane);
         if (phys < 0 || phys >= a.num_blocks) {
           raise_flag(a.status, PA_FLAG_BLOCK_RANGE);
           phys = -1;
@@ -360,10 +367,10 @@ __global__ void __launch_bounds__(192, 1)
           l_t[h] = 0.f;
         }
         L = __ldg(a.context_lens + g.s);
-        lim = min(L, g.bhi * BS);  // tokens this CTA owns end here
+        lim = min(L, (g.skip + g.bhi) * BS);  // tokens this CTA owns end here
         row = __ldg(a.query_start_loc + g.s);
       }
-      const int tok = it.tb * BS + tid;
+      const int tok = (g.skip + it.tb) * BS + tid;
       const bool valid = tok < lim;
       failed = failed || !mbar_wait(&s_full[b], (i >> 1) & 1, a.status);
       failed = __any_sync(0xffffffffu, failed);

@@ -275,6 +275,35 @@ pa_status pa_copy_blocks(const int32_t* src_dst_pairs, int32_t num_pairs, void* 
 }
 
 namespace {
+// Encode the decode tensor maps and launch the decode grid (tensor-core kernel
+// for grouped bf16 heads of 128, CUDA-core kernel otherwise). *e receives the
+// launch status; the return value reports a tensor-map failure.
+pa_status launch_decode_path(DecodeArgs& a, const void* q, const void* k_cache, const void* v_cache,
+                             int32_t num_q_heads, int32_t num_q_tokens, const pa_cache_desc* cache,
+                             cudaStream_t s, cudaError_t* e) {
+  pa_status st;
+  const int32_t group = num_q_heads / cache->num_kv_heads;
+  // q as a 3-D tensor {head_dim, num_q_heads, num_q_tokens}
+  const uint64_t qd[3] = {uint64_t(cache->head_dim), uint64_t(num_q_heads), uint64_t(num_q_tokens)};
+  const uint64_t qs[2] = {uint64_t(cache->head_dim) * 2, uint64_t(num_q_heads) * cache->head_dim * 2};
+  CUtensorMap kmap, vmap;
+  if (decode_uses_tc(group, *cache)) {
+    // tensor-core decode: 64-column (128-byte) swizzled boxes, Q^T per KV head
+    CUtensorMap qmap;
+    const uint32_t qbox[3] = {64, uint32_t(group), 1};
+    if ((st = tensor_map(&qmap, q, 3, qd, qs, qbox, PA_BF16, 128)) != PA_OK) return st;
+    if ((st = cache_map(&kmap, k_cache, *cache, 64, 128)) != PA_OK) return st;
+    if ((st = cache_map(&vmap, v_cache, *cache, 64, 128)) != PA_OK) return st;
+    *e = launch_decode_tc(a, qmap, kmap, vmap, *cache, s);
+  } else {
+    const uint32_t kh = decode_kv_heads_per_cta(group, *cache);
+    if ((st = cache_map(&kmap, k_cache, *cache, cache->head_dim, 0, kh)) != PA_OK) return st;
+    if ((st = cache_map(&vmap, v_cache, *cache, cache->head_dim, 0, kh)) != PA_OK) return st;
+    *e = launch_decode(a, kmap, vmap, *cache, s);
+  }
+  return PA_OK;
+}
+
 // Workspace layout of one call: partial outputs, their log-sum-exp, and the
 // per-sequence decode block prefix. False for arguments the size query cannot use.
 struct WorkspaceLayout {
@@ -367,26 +396,16 @@ pa_status pa_attention(const void* q, const void* k_cache, const void* v_cache,
   a.max_context_len = max_context_len;
   a.grid = 0;
   a.scale_log2 = scale_log2;
+  a.skip_blocks = nullptr;
+  a.l1_o = nullptr;
+  a.l1_lse = nullptr;
+  a.l1_max_chunks = 0;
+  a.l1_chunk_blocks = 1;
 
   const int32_t group = num_q_heads / cache->num_kv_heads;
-  // q as a 3-D tensor {head_dim, num_q_heads, num_q_tokens} (decode and prefill maps)
   const uint64_t qd[3] = {uint64_t(cache->head_dim), uint64_t(num_q_heads), uint64_t(num_q_tokens)};
   const uint64_t qs[2] = {uint64_t(cache->head_dim) * 2, uint64_t(num_q_heads) * cache->head_dim * 2};
-  CUtensorMap kmap, vmap;
-  if (decode_uses_tc(group, *cache)) {
-    // tensor-core decode: 64-column (128-byte) swizzled boxes, Q^T per KV head
-    CUtensorMap qmap;
-    const uint32_t qbox[3] = {64, uint32_t(group), 1};
-    if ((st = tensor_map(&qmap, q, 3, qd, qs, qbox, PA_BF16, 128)) != PA_OK) return st;
-    if ((st = cache_map(&kmap, k_cache, *cache, 64, 128)) != PA_OK) return st;
-    if ((st = cache_map(&vmap, v_cache, *cache, 64, 128)) != PA_OK) return st;
-    e = launch_decode_tc(a, qmap, kmap, vmap, *cache, s);
-  } else {
-    const uint32_t kh = decode_kv_heads_per_cta(group, *cache);
-    if ((st = cache_map(&kmap, k_cache, *cache, cache->head_dim, 0, kh)) != PA_OK) return st;
-    if ((st = cache_map(&vmap, v_cache, *cache, cache->head_dim, 0, kh)) != PA_OK) return st;
-    e = launch_decode(a, kmap, vmap, *cache, s);
-  }
+  if ((st = launch_decode_path(a, q, k_cache, v_cache, num_q_heads, num_q_tokens, cache, s, &e)) != PA_OK) return st;
   if (e != cudaSuccess) return cuda_fail(e, "decode launch");
   e = launch_decode_combine(a, *cache, s);
   if (e != cudaSuccess) return cuda_fail(e, "decode combine launch");
@@ -406,6 +425,13 @@ pa_status pa_attention(const void* q, const void* k_cache, const void* v_cache,
     p.max_query_len = max_query_len;
     p.num_q_tokens = num_q_tokens;
     p.scale_log2 = scale_log2;
+    p.groups = nullptr;
+    p.skip_blocks = nullptr;
+    p.num_groups = 0;
+    p.l1_o = nullptr;
+    p.l1_lse = nullptr;
+    p.l1_max_chunks = 0;
+    p.l1_chunk_blocks = 1;
     // K/V boxes are 64 columns wide (128 bytes) to match the 128-byte swizzle
     // of the MMA tiles.
     const int32_t gh = prefill_heads_per_tile(group);
@@ -418,6 +444,157 @@ pa_status pa_attention(const void* q, const void* k_cache, const void* v_cache,
     if (e == cudaErrorNotSupported) return fail(PA_ERR_UNSUPPORTED, "prefill rows not supported yet");
     if (e != cudaSuccess) return cuda_fail(e, "prefill launch");
   }
+  return PA_OK;
+}
+
+}  // extern "C"
+
+namespace {
+// Cascade decode: the prefix pass splits each group's shared blocks into
+// chunks of this many tokens (one work item per chunk and member tile).
+constexpr int32_t kCascadeChunkTokens = 256;
+int32_t cascade_chunk_blocks(const pa_cache_desc& c) { return kCascadeChunkTokens / c.block_size; }
+int32_t cascade_max_chunks(int32_t max_shared_blocks, const pa_cache_desc& c) {
+  return ceil_div(max_shared_blocks, cascade_chunk_blocks(c));
+}
+struct CascadeLayout {
+  WorkspaceLayout base;
+  size_t l1_o_off = 0, l1_lse_off = 0, bytes = 0;
+};
+bool cascade_layout(int32_t num_seqs, int32_t num_q_heads, int32_t max_context_len, int32_t max_shared_blocks,
+                    const pa_cache_desc* cache, CascadeLayout* w) {
+  if (!workspace_layout(num_seqs, num_q_heads, 1, max_context_len, cache, &w->base) || max_shared_blocks < 0)
+    return false;
+  if (num_seqs == 0) return true;
+  const size_t rows = size_t(num_seqs) * num_q_heads * size_t(cascade_max_chunks(max_shared_blocks, *cache));
+  w->l1_o_off = (w->base.bytes + 255) & ~size_t(255);
+  w->l1_lse_off = (w->l1_o_off + rows * cache->head_dim * 4 + 255) & ~size_t(255);
+  w->bytes = w->l1_lse_off + rows * 4;
+  return true;
+}
+}  // namespace
+
+extern "C" {
+
+size_t pa_attention_cascade_workspace_size(int32_t num_seqs, int32_t num_q_heads, int32_t max_context_len,
+                                           int32_t max_shared_blocks, const pa_cache_desc* cache) {
+  CascadeLayout w;
+  if (!cascade_layout(num_seqs, num_q_heads, max_context_len, max_shared_blocks, cache, &w)) return 0;
+  return w.bytes;
+}
+
+pa_status pa_attention_cascade(const void* q, const void* k_cache, const void* v_cache,
+                               const int32_t* block_tables, int32_t max_blocks_per_seq,
+                               const int32_t* context_lens, const int32_t* query_start_loc, int32_t num_seqs,
+                               int32_t num_q_heads, int32_t max_context_len, const int32_t* shared_blocks,
+                               const int32_t* groups, int32_t num_groups, int32_t max_group_size,
+                               int32_t max_shared_blocks, float scale, const pa_cache_desc* cache, void* out,
+                               void* workspace, size_t workspace_bytes, void* stream) {
+  pa_status st = check_cache(cache);
+  if (st != PA_OK) return st;
+  if (num_seqs < 0 || max_context_len < 0 || num_groups < 0 || max_group_size < 0 || max_shared_blocks < 0)
+    return fail(PA_ERR_INVALID_ARG, "pa_attention_cascade: negative size argument");
+  if (num_q_heads < 1 || num_q_heads % cache->num_kv_heads)
+    return fail(PA_ERR_INVALID_ARG, "num_q_heads %d must be a positive multiple of num_kv_heads %d",
+                num_q_heads, cache->num_kv_heads);
+  if (max_blocks_per_seq < 1) return fail(PA_ERR_INVALID_ARG, "max_blocks_per_seq must be >= 1");
+  if (num_seqs == 0) return PA_OK;
+  if (cache->dtype != PA_BF16) return fail(PA_ERR_UNSUPPORTED, "cascade decode needs a bf16 cache");
+  if (num_groups > num_seqs) return fail(PA_ERR_INVALID_ARG, "more groups than sequences");
+  if (num_groups > 0 && (!shared_blocks || !groups || max_group_size < 1 || max_shared_blocks < 1))
+    return fail(PA_ERR_INVALID_ARG, "groups need shared_blocks, groups and positive bounds");
+  if (max_shared_blocks > max_blocks_per_seq)
+    return fail(PA_ERR_INVALID_ARG, "max_shared_blocks %d > max_blocks_per_seq %d", max_shared_blocks,
+                max_blocks_per_seq);
+  if (!q || !k_cache || !v_cache || !block_tables || !context_lens || !query_start_loc || !out)
+    return fail(PA_ERR_INVALID_ARG, "pa_attention_cascade: NULL pointer argument");
+  if (!aligned16(q) || !aligned16(out) || !aligned16(k_cache) || !aligned16(v_cache))
+    return fail(PA_ERR_INVALID_ARG, "pa_attention_cascade: q, out and caches must be 16-byte aligned");
+  if (num_seqs > kMaxSeqs) return fail(PA_ERR_UNSUPPORTED, "num_seqs %d > %d", num_seqs, kMaxSeqs);
+  if (int64_t(max_blocks_per_seq) * cache->block_size > (1ll << 30))
+    return fail(PA_ERR_UNSUPPORTED, "max_blocks_per_seq too large");
+  if (!(scale == scale)) return fail(PA_ERR_INVALID_ARG, "scale is NaN");
+  CascadeLayout wl;
+  cascade_layout(num_seqs, num_q_heads, max_context_len, num_groups > 0 ? max_shared_blocks : 0, cache, &wl);
+  if (!workspace || workspace_bytes < wl.bytes)
+    return fail(PA_ERR_INVALID_ARG, "workspace of %zu bytes needed, %zu given", wl.bytes,
+                workspace ? workspace_bytes : size_t(0));
+  if (!aligned16(workspace)) return fail(PA_ERR_INVALID_ARG, "workspace must be 16-byte aligned");
+
+  unsigned* status = nullptr;
+  cudaError_t e = status_ptr(&status);
+  if (e != cudaSuccess) return cuda_fail(e, "status word");
+  const cudaStream_t s = static_cast<cudaStream_t>(stream);
+  const float scale_log2 = static_cast<float>(double(scale) * 1.4426950408889634);
+  char* ws = static_cast<char*>(workspace);
+  const int32_t chunk_blocks = cascade_chunk_blocks(*cache);
+  const int32_t max_chunks = num_groups > 0 ? cascade_max_chunks(max_shared_blocks, *cache) : 0;
+
+  DecodeArgs a;
+  a.q = q;
+  a.out = out;
+  a.block_tables = block_tables;
+  a.context_lens = context_lens;
+  a.query_start_loc = query_start_loc;
+  a.part_o = reinterpret_cast<float*>(ws);
+  a.part_lse = reinterpret_cast<float*>(ws + wl.base.lse_off);
+  a.seq_prefix = reinterpret_cast<int32_t*>(ws + wl.base.prefix_off);
+  a.status = status;
+  a.max_blocks_per_seq = max_blocks_per_seq;
+  a.num_seqs = num_seqs;
+  a.num_q_heads = num_q_heads;
+  a.num_kv_heads = cache->num_kv_heads;
+  a.num_blocks = cache->num_blocks;
+  a.max_context_len = max_context_len;
+  a.grid = 0;
+  a.scale_log2 = scale_log2;
+  a.skip_blocks = num_groups > 0 ? shared_blocks : nullptr;
+  a.l1_o = reinterpret_cast<float*>(ws + wl.l1_o_off);
+  a.l1_lse = reinterpret_cast<float*>(ws + wl.l1_lse_off);
+  a.l1_max_chunks = max_chunks;
+  a.l1_chunk_blocks = chunk_blocks;
+
+  // 1. every sequence's own blocks (past its group's shared ones): partials
+  if ((st = launch_decode_path(a, q, k_cache, v_cache, num_q_heads, num_seqs, cache, s, &e)) != PA_OK) return st;
+  if (e != cudaSuccess) return cuda_fail(e, "decode launch");
+  // 2. each group's shared blocks, read once for all its members: partials
+  if (num_groups > 0) {
+    PrefillArgs p;
+    p.out = out;
+    p.block_tables = block_tables;
+    p.context_lens = context_lens;
+    p.query_start_loc = query_start_loc;
+    p.status = status;
+    p.max_blocks_per_seq = max_blocks_per_seq;
+    p.num_seqs = num_seqs;
+    p.num_q_heads = num_q_heads;
+    p.num_kv_heads = cache->num_kv_heads;
+    p.num_blocks = cache->num_blocks;
+    p.max_context_len = max_context_len;
+    p.max_query_len = max_group_size;
+    p.num_q_tokens = num_seqs;
+    p.scale_log2 = scale_log2;
+    p.groups = groups;
+    p.skip_blocks = shared_blocks;
+    p.num_groups = num_groups;
+    p.l1_o = reinterpret_cast<float*>(ws + wl.l1_o_off);
+    p.l1_lse = reinterpret_cast<float*>(ws + wl.l1_lse_off);
+    p.l1_max_chunks = max_chunks;
+    p.l1_chunk_blocks = chunk_blocks;
+    const int32_t gh = prefill_heads_per_tile(num_q_heads / cache->num_kv_heads);
+    const uint64_t qd[3] = {uint64_t(cache->head_dim), uint64_t(num_q_heads), uint64_t(num_seqs)};
+    const uint64_t qs[2] = {uint64_t(cache->head_dim) * 2, uint64_t(num_q_heads) * cache->head_dim * 2};
+    const uint32_t qbox[3] = {64, uint32_t(gh), uint32_t(128 / gh)};
+    CUtensorMap qmap, pk, pv;
+    if ((st = tensor_map(&qmap, q, 3, qd, qs, qbox, PA_BF16, 128)) != PA_OK) return st;
+    if ((st = cache_map(&pk, k_cache, *cache, 64, 128)) != PA_OK) return st;
+    if ((st = cache_map(&pv, v_cache, *cache, 64, 128)) != PA_OK) return st;
+    e = launch_cascade_prefix(p, qmap, pk, pv, *cache, s);
+    if (e != cudaSuccess) return cuda_fail(e, "cascade prefix launch");
+  }
+  // 3. merge: the prefix grid finishes no earlier than the decode grid
+  e = launch_decode_combine(a, *cache, s);
+  if (e != cudaSuccess) return cuda_fail(e, "decode combine launch");
   return PA_OK;
 }
 

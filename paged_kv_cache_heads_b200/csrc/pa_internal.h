@@ -30,6 +30,12 @@ struct DecodeArgs {
   int32_t max_context_len;
   int32_t grid;         // CTAs of the decode grid (set by launch_decode)
   float scale_log2;     // scale * log2(e)
+  // Cascade (shared-prefix) decode; all null / 0 otherwise.
+  const int32_t* skip_blocks;  // [num_seqs] leading table blocks read by the prefix pass instead
+  const float* l1_o;           // [num_seqs * num_q_heads * l1_max_chunks][head_dim] prefix-pass partials
+  const float* l1_lse;         // [num_seqs * num_q_heads * l1_max_chunks]
+  int32_t l1_max_chunks;       // prefix chunks per sequence and head (slot stride)
+  int32_t l1_chunk_blocks;     // blocks per prefix chunk
 };
 
 struct PrefillArgs {
@@ -47,6 +53,15 @@ struct PrefillArgs {
   int32_t max_query_len;
   int32_t num_q_tokens;
   float scale_log2;
+  // Cascade prefix pass (kernel instantiated with the cascade flag): work
+  // items run over the groups' shared blocks instead of the prefill rows.
+  const int32_t* groups;       // [num_groups][2]: first member sequence, member count
+  const int32_t* skip_blocks;  // [num_seqs] shared blocks of each member (same within a group)
+  int32_t num_groups;
+  float* l1_o;                 // partial outputs, slot ((s * num_q_heads + h) * l1_max_chunks + chunk)
+  float* l1_lse;
+  int32_t l1_max_chunks;
+  int32_t l1_chunk_blocks;
 };
 
 // Sets the calling thread's pa_last_error() message.
@@ -76,6 +91,9 @@ cudaError_t launch_decode_tc(DecodeArgs& a, const CUtensorMap& qmap, const CUten
 cudaError_t launch_decode_combine(const DecodeArgs& a, const pa_cache_desc& c, cudaStream_t stream);
 cudaError_t launch_prefill(const PrefillArgs& a, const CUtensorMap& qmap, const CUtensorMap& kmap,
                            const CUtensorMap& vmap, const pa_cache_desc& c, cudaStream_t stream);
+// The prefix pass of cascade decode (same kernel, cascade items, partial output).
+cudaError_t launch_cascade_prefix(const PrefillArgs& a, const CUtensorMap& qmap, const CUtensorMap& kmap,
+                                  const CUtensorMap& vmap, const pa_cache_desc& c, cudaStream_t stream);
 
 // Query heads packed into one 128-row prefill tile (the rest of its rows are tokens).
 int32_t prefill_heads_per_tile(int32_t group);

@@ -87,9 +87,10 @@ __device__ __forceinline__ int prefill_scan(int x, int* warp_tot, int& total) {
 
 struct Item {
   int s, r0, q_len, L, t0, hq0, hk, ntile;
+  int kb0, chunk;  // cascade prefix pass: first key block of the item's chunk, and its index
 };
 
-template <int D, int BS, int GH>
+template <int D, int BS, int GH, bool CASC>
 __global__ void __launch_bounds__(160, 2)
     paged_prefill_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constant__ CUtensorMap kmap,
                          const __grid_constant__ CUtensorMap vmap, const PrefillArgs a) {
@@ -138,10 +139,13 @@ __global__ void __launch_bounds__(160, 2)
   // ---- tiles of every prefill sequence
   int carry = 0;
   if (tid == 0) prefix[0] = 0;
-  for (int base = 0; base < a.num_seqs; base += blockDim.x) {
+  // Items: (sequence, 128-row tile, head group) over the prefill rows; in the
+  // cascade prefix pass (group, chunk of shared blocks, member tile, head group)
+  const int n_src = CASC ? a.num_groups : a.num_seqs;
+  for (int base = 0; base < n_src; base += blockDim.x) {
     const int s = base + tid;
     int n = 0;
-    if (s < a.num_seqs) {
+    if (s < n_src && !CASC) {
       const int L = __ldg(a.context_lens + s);
       const int r0 = __ldg(a.query_start_loc + s);
       const int ql = __ldg(a.query_start_loc + s + 1) - r0;
@@ -155,38 +159,74 @@ __global__ void __launch_bounds__(160, 2)
           n = ((ql + C::kTOK - 1) / C::kTOK) * HGp;
         }
       }
+    } else if (s < n_src) {
+      // group s: members lead .. lead + m - 1 (one decode row each, rows r0 ..),
+      // sharing the first nb blocks of the leader's table
+      const int lead = __ldg(a.groups + 2 * s);
+      const int m = __ldg(a.groups + 2 * s + 1);
+      const int nb = m > 0 && lead >= 0 && lead + m <= a.num_seqs ? __ldg(a.skip_blocks + lead) : 0;
+      const int r0 = nb > 0 ? __ldg(a.query_start_loc + lead) : 0;
+      clen[s] = nb;
+      qrow[s] = r0;
+      if (m > 0) {
+        if (nb < 1 || lead < 0 || lead + m > a.num_seqs || nb * BS > __ldg(a.context_lens + lead) || r0 < 0 ||
+            r0 + m > a.num_q_tokens) {
+          raise_flag(a.status, PA_FLAG_CONTEXT_RANGE);
+        } else {
+          n = ((nb + a.l1_chunk_blocks - 1) / a.l1_chunk_blocks) * ((m + C::kTOK - 1) / C::kTOK) * HGp;
+        }
+      }
     }
     int total;
     const int incl = prefill_scan(n, warp_tot, total);
-    if (s < a.num_seqs) prefix[s + 1] = carry + incl;
+    if (s < n_src) prefix[s + 1] = carry + incl;
     carry += total;
   }
   tc::fence_before_sync();
   __syncthreads();
   tc::fence_after_sync();
   const uint32_t tmem = *tmem_slot;
-  const int W = prefix[a.num_seqs];
+  const int W = prefix[n_src];
 
   auto item_of = [&](int w) {
-    int lo = 0, hi = a.num_seqs;
+    int lo = 0, hi = n_src;
     while (hi - lo > 1) {
       const int mid = (lo + hi) >> 1;
       if (prefix[mid] <= w) lo = mid; else hi = mid;
     }
     Item it;
-    it.s = lo;
     const int r = w - prefix[lo];
-    const int mt = r / HGp;
-    const int hg = r - mt * HGp;
+    const int mt0 = r / HGp;
+    const int hg = r - mt0 * HGp;
     it.r0 = qrow[lo];
-    it.L = clen[lo];
-    it.q_len = 0;
-    it.t0 = mt * C::kTOK;
     it.hq0 = hg * GH;
     it.hk = it.hq0 / G;
+    if (!CASC) {
+      it.s = lo;
+      it.L = clen[lo];
+      it.q_len = 0;
+      it.t0 = mt0 * C::kTOK;
+      it.kb0 = 0;
+      it.chunk = 0;
+    } else {
+      // mt0 = chunk * member_tiles + member tile
+      const int lead = __ldg(a.groups + 2 * lo);
+      const int m = __ldg(a.groups + 2 * lo + 1);
+      const int mtiles = (m + C::kTOK - 1) / C::kTOK;
+      it.s = lead;
+      it.q_len = m;
+      it.chunk = mt0 / mtiles;
+      it.t0 = (mt0 - it.chunk * mtiles) * C::kTOK;
+      it.kb0 = it.chunk * a.l1_chunk_blocks;
+      it.L = min(a.l1_chunk_blocks, clen[lo] - it.kb0) * BS;  // keys of this chunk
+    }
     return it;
   };
   auto finish_item = [&](Item& it) {
+    if (CASC) {  // every member row sees every key of the chunk
+      it.ntile = (it.L + kBN - 1) / kBN;
+      return;
+    }
     it.q_len = __ldg(a.query_start_loc + it.s + 1) - it.r0;
     const int t_last = min(it.t0 + C::kTOK, it.q_len) - 1;
     const int p_max = it.L - it.q_len + t_last;
@@ -218,7 +258,7 @@ __global__ void __launch_bounds__(160, 2)
             const int lb = j * C::kBlocksPerTile + b;
             int phys = -1;
             if (lb < nblk_valid) {
-              phys = __ldg(row + lb);
+              phys = __ldg(row + it.kb0 + lb);
               if (phys < 0 || phys >= a.num_blocks) {
                 raise_flag(a.status, PA_FLAG_BLOCK_RANGE);
                 phys = -1;
@@ -246,7 +286,8 @@ __global__ void __launch_bounds__(160, 2)
     Item it = item_of(w);
     finish_item(it);
     const int tok = it.t0 + r / GH;
-    const int lim = min(it.L - it.q_len + tok, it.L - 1);  // last key this row may see
+    // last key this row may see (the whole chunk in the cascade prefix pass)
+    const int lim = CASC ? it.L - 1 : min(it.L - it.q_len + tok, it.L - 1);
     float m_used = -CUDART_INF_F, l = 0.f;
     mbar_wait(q_full, it_no & 1, a.status);
     for (int j = 0; j < it.ntile; ++j, ++gj) {
@@ -354,12 +395,22 @@ __global__ void __launch_bounds__(160, 2)
     const bool row_ok = tok < it.q_len;
     __nv_bfloat16* orow = static_cast<__nv_bfloat16*>(a.out) +
                           (static_cast<size_t>(it.r0 + tok) * a.num_q_heads + it.hq0 + r % GH) * D;
+    // cascade prefix pass: partial (O / l, log2-sum-exp) of member it.s + tok, this chunk
+    const size_t l1_slot =
+        (static_cast<size_t>(it.s + tok) * a.num_q_heads + it.hq0 + r % GH) * a.l1_max_chunks + it.chunk;
+    if (CASC && row_ok) a.l1_lse[l1_slot] = m_used + log2f(l);
 #pragma unroll 1
     for (int q = 0; q < D / 32; ++q) {
       float ov[32];
       tc::ld32(t_lane + o_col + 32 * q, ov);
       tc::wait_ld();
-      if (row_ok) {
+      if (CASC && row_ok) {
+        float* po = a.l1_o + l1_slot * D + 32 * q;
+#pragma unroll
+        for (int v4 = 0; v4 < 8; ++v4)
+          *reinterpret_cast<float4*>(po + 4 * v4) = make_float4(ov[4 * v4] * inv_l, ov[4 * v4 + 1] * inv_l,
+                                                                ov[4 * v4 + 2] * inv_l, ov[4 * v4 + 3] * inv_l);
+      } else if (row_ok) {
 #pragma unroll
         for (int v4 = 0; v4 < 4; ++v4) {
           uint32_t pk[4];
@@ -382,11 +433,11 @@ __global__ void __launch_bounds__(160, 2)
   if (tid == 0) grid_dependency_wait();  // finish no earlier than the previous grid
 }
 
-template <int D, int BS, int GH>
+template <int D, int BS, int GH, bool CASC>
 cudaError_t launch_prefill_t(const PrefillArgs& a, const CUtensorMap& qmap, const CUtensorMap& kmap,
                              const CUtensorMap& vmap, cudaStream_t stream) {
   using C = PrefillCfg<D, BS, GH>;
-  auto kern = paged_prefill_kernel<D, BS, GH>;
+  auto kern = paged_prefill_kernel<D, BS, GH, CASC>;
   const size_t smem = C::smem_bytes(a.num_seqs);
   static int configured_smem[64] = {0};
   int dev = 0;
@@ -404,37 +455,39 @@ cudaError_t launch_prefill_t(const PrefillArgs& a, const CUtensorMap& qmap, cons
   }
   // TMEM holds 512 columns per SM; each CTA allocates kTmemCols of them.
   const int per_sm = ctas_per_sm(reinterpret_cast<const void*>(kern), 160, smem, 512 / C::kTmemCols);
-  const int64_t bound = static_cast<int64_t>(a.num_seqs) * (a.num_q_heads / GH) *
-                        ((a.max_query_len + C::kTOK - 1) / C::kTOK);
+  // max_query_len bounds the rows of a sequence (prefill) or the members of a
+  // group (cascade); in the cascade pass each group also has its chunks
+  const int64_t rows = CASC ? static_cast<int64_t>(a.num_groups) * a.l1_max_chunks : a.num_seqs;
+  const int64_t bound = rows * (a.num_q_heads / GH) * ((a.max_query_len + C::kTOK - 1) / C::kTOK);
   const int64_t slots = static_cast<int64_t>(num_sms()) * per_sm;
   const int grid = static_cast<int>(bound < slots ? (bound > 0 ? bound : 1) : slots);
   // Chained launch: the prefill rows do not read anything the decode grid
   // writes, so this grid may start as soon as SMs free up; each CTA waits for
   // the previous grid before it exits, which keeps stream order for whatever
   // is launched after pa_attention.
-  log_launch("paged_prefill_kernel", grid, 160, smem, per_sm);
+  log_launch(CASC ? "paged_prefill_kernel(cascade prefix)" : "paged_prefill_kernel", grid, 160, smem, per_sm);
   return launch_chained(kern, dim3(grid), dim3(160), smem, stream, qmap, kmap, vmap, a);
 }
 
-template <int D, int BS>
+template <int D, int BS, bool CASC>
 cudaError_t launch_prefill_gh(const PrefillArgs& a, const CUtensorMap& qmap, const CUtensorMap& kmap,
                               const CUtensorMap& vmap, int gh, cudaStream_t stream) {
   switch (gh) {
-    case 16: return launch_prefill_t<D, BS, 16>(a, qmap, kmap, vmap, stream);
-    case 8: return launch_prefill_t<D, BS, 8>(a, qmap, kmap, vmap, stream);
-    case 4: return launch_prefill_t<D, BS, 4>(a, qmap, kmap, vmap, stream);
-    case 2: return launch_prefill_t<D, BS, 2>(a, qmap, kmap, vmap, stream);
-    default: return launch_prefill_t<D, BS, 1>(a, qmap, kmap, vmap, stream);
+    case 16: return launch_prefill_t<D, BS, 16, CASC>(a, qmap, kmap, vmap, stream);
+    case 8: return launch_prefill_t<D, BS, 8, CASC>(a, qmap, kmap, vmap, stream);
+    case 4: return launch_prefill_t<D, BS, 4, CASC>(a, qmap, kmap, vmap, stream);
+    case 2: return launch_prefill_t<D, BS, 2, CASC>(a, qmap, kmap, vmap, stream);
+    default: return launch_prefill_t<D, BS, 1, CASC>(a, qmap, kmap, vmap, stream);
   }
 }
 
-template <int D>
+template <int D, bool CASC>
 cudaError_t launch_prefill_bs(const PrefillArgs& a, const CUtensorMap& qmap, const CUtensorMap& kmap,
                               const CUtensorMap& vmap, int bs, int gh, cudaStream_t stream) {
   switch (bs) {
-    case 8: return launch_prefill_gh<D, 8>(a, qmap, kmap, vmap, gh, stream);
-    case 16: return launch_prefill_gh<D, 16>(a, qmap, kmap, vmap, gh, stream);
-    default: return launch_prefill_gh<D, 32>(a, qmap, kmap, vmap, gh, stream);
+    case 8: return launch_prefill_gh<D, 8, CASC>(a, qmap, kmap, vmap, gh, stream);
+    case 16: return launch_prefill_gh<D, 16, CASC>(a, qmap, kmap, vmap, gh, stream);
+    default: return launch_prefill_gh<D, 32, CASC>(a, qmap, kmap, vmap, gh, stream);
   }
 }
 
@@ -448,8 +501,16 @@ cudaError_t launch_prefill(const PrefillArgs& a, const CUtensorMap& qmap, const 
                            const CUtensorMap& vmap, const pa_cache_desc& c, cudaStream_t stream) {
   if (c.dtype != PA_BF16) return cudaErrorNotSupported;
   const int gh = prefill_heads_per_tile(a.num_q_heads / a.num_kv_heads);
-  if (c.head_dim == 64) return launch_prefill_bs<64>(a, qmap, kmap, vmap, c.block_size, gh, stream);
-  return launch_prefill_bs<128>(a, qmap, kmap, vmap, c.block_size, gh, stream);
+  if (c.head_dim == 64) return launch_prefill_bs<64, false>(a, qmap, kmap, vmap, c.block_size, gh, stream);
+  return launch_prefill_bs<128, false>(a, qmap, kmap, vmap, c.block_size, gh, stream);
+}
+
+cudaError_t launch_cascade_prefix(const PrefillArgs& a, const CUtensorMap& qmap, const CUtensorMap& kmap,
+                                  const CUtensorMap& vmap, const pa_cache_desc& c, cudaStream_t stream) {
+  if (c.dtype != PA_BF16) return cudaErrorNotSupported;
+  const int gh = prefill_heads_per_tile(a.num_q_heads / a.num_kv_heads);
+  if (c.head_dim == 64) return launch_prefill_bs<64, true>(a, qmap, kmap, vmap, c.block_size, gh, stream);
+  return launch_prefill_bs<128, true>(a, qmap, kmap, vmap, c.block_size, gh, stream);
 }
 
 }  // namespace pa

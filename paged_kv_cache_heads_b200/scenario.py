@@ -19,8 +19,8 @@ from dataclasses import dataclass, field
 import numpy as np
 import torch
 
-from . import BlockManager, CacheDesc, PA_BF16, PA_FP32, pa_attention, pa_attention_workspace_size, \
-    pa_copy_blocks, pa_store_kv
+from . import BlockManager, CacheDesc, PA_BF16, PA_FP32, pa_attention, pa_attention_cascade, \
+    pa_attention_cascade_workspace_size, pa_attention_workspace_size, pa_copy_blocks, pa_store_kv
 from . import workloads as W
 
 
@@ -176,3 +176,39 @@ def capture_step(b: DeviceBatch, pre=None, post=None):
         if post is not None:
             post()
     return g
+
+
+@dataclass
+class CascadePlan:
+    shared_blocks: torch.Tensor   # int32 [S]
+    groups: torch.Tensor          # int32 [G, 2] (first, count)
+    num_groups: int
+    max_group_size: int
+    max_shared_blocks: int
+    workspace: torch.Tensor
+    host: dict = field(default_factory=dict)
+
+
+def plan_cascade(b: DeviceBatch, min_shared_blocks: int = 1) -> CascadePlan:
+    """Groups of b's batch that share leading blocks (from the library's block
+    manager) and a workspace for pa_attention_cascade."""
+    shared, groups = b.host["bm"].cascade_groups(b.wl.batch_seqs, min_shared_blocks)
+    dev = b.q.device
+    ng = int(groups.shape[0])
+    mg = int(groups[:, 1].max()) if ng else 0
+    ms = int(shared.max()) if shared.size else 0
+    ws_bytes = pa_attention_cascade_workspace_size(len(b.wl.batch_seqs), b.wl.geometry.num_q_heads,
+                                                   b.max_context_len, ms, b.desc)
+    ws = torch.empty(max(ws_bytes, 16), dtype=torch.uint8, device=dev)
+    g = torch.from_numpy(np.ascontiguousarray(groups if ng else np.zeros((1, 2), np.int32))).to(dev)
+    return CascadePlan(torch.from_numpy(np.ascontiguousarray(shared)).to(dev), g, ng, mg, ms, ws,
+                       dict(shared=shared, groups=groups))
+
+
+def run_attention_cascade(b: DeviceBatch, plan: CascadePlan, stream=None, out=None):
+    geo = b.wl.geometry
+    pa_attention_cascade(b.q, b.k_cache, b.v_cache, b.block_tables, geo.max_blocks_per_seq, b.context_lens,
+                         b.query_start_loc, len(b.wl.batch_seqs), geo.num_q_heads, b.max_context_len,
+                         plan.shared_blocks, plan.groups, plan.num_groups, plan.max_group_size,
+                         plan.max_shared_blocks, b.wl.scale, b.desc, b.out if out is None else out,
+                         plan.workspace, stream=stream)

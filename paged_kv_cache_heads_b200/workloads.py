@@ -276,6 +276,53 @@ def random_case(seed: int, *, num_seqs: int, q_lens, ctx_extra, num_kv_heads: in
                     notes=dict(context_lens=lens))
 
 
+def shared_prefix_case(seed: int, *, groups, singles, num_kv_heads: int, group: int, head_dim: int,
+                       block_size: int, dtype: str, max_blocks_per_seq: int | None = None) -> Workload:
+    """Decode batch with shared prefixes, for cascade parity.
+
+    ``groups`` is a list of ``(prefix_len, [L_1, L_2, ...])``: the first member
+    holds the prefix, the others fork it whole, and member i grows to L_i
+    tokens (L_i > prefix_len; the last token is the step's decode row).
+    ``singles`` are lengths of sequences that share nothing; they are placed
+    between the groups (batch order: single, group 0, single, group 1, ...).
+    """
+    draw = _Draw(seed)
+    hkv, d = num_kv_heads, head_dim
+    order, lens, ops = [], [], []
+    sid = 0
+    singles = list(singles)
+    for gi, (plen, member_lens) in enumerate(groups):
+        if singles:
+            L = int(singles.pop(0))
+            ops.append(Op("add", sid, L - 1, k=draw.rows(L - 1, hkv, d, dtype), v=draw.rows(L - 1, hkv, d, dtype)))
+            order.append(sid)
+            lens.append(L)
+            sid += 1
+        lead = sid
+        ops.append(Op("add", lead, plen, k=draw.rows(plen, hkv, d, dtype), v=draw.rows(plen, hkv, d, dtype)))
+        for m, L in enumerate(member_lens):
+            if m:
+                ops.append(Op("fork", sid, plen, parent=lead))
+            n = int(L) - plen - 1
+            ops.append(Op("append", sid, n, k=draw.rows(n, hkv, d, dtype), v=draw.rows(n, hkv, d, dtype)))
+            order.append(sid)
+            lens.append(int(L))
+            sid += 1
+    for L in singles:
+        ops.append(Op("add", sid, L - 1, k=draw.rows(L - 1, hkv, d, dtype), v=draw.rows(L - 1, hkv, d, dtype)))
+        order.append(sid)
+        lens.append(int(L))
+        sid += 1
+    for s in order:
+        ops.append(Op("append", s, 1, k=draw.rows(1, hkv, d, dtype), v=draw.rows(1, hkv, d, dtype)))
+    nb = sum(-(-L // block_size) for L in lens) + 8 * len(lens) + 8
+    mb = max_blocks_per_seq or max(-(-L // block_size) for L in lens)
+    geo = Geometry(nb, block_size, hkv, hkv * group, d, dtype, mb)
+    q = draw.rows(len(order), hkv * group, d, dtype)
+    return Workload("shared_prefix_%d" % seed, geo, draw.pool_order(nb), ops, order, [1] * len(order), q,
+                    1.0 / math.sqrt(d), step_ops=len(order), notes=dict(context_lens=lens))
+
+
 CONFIGS = {
     "tiny": tiny,
     "llama7b": llama7b_decode,

@@ -293,3 +293,55 @@ def test_compaction_matches_oracle_on_workloads():
         pa_, pb = a.compact(), b.compact()
         assert pa_ == pb and len(pa_) > 0
         _same_state(a, b, live)
+
+
+@pytest.mark.parametrize("seed", range(6))
+def test_cascade_groups_match_oracle(seed):
+    rng = np.random.default_rng(900 + seed)
+    bs = int(rng.choice([8, 16, 32]))
+    groups = [(int(rng.integers(1, 6 * bs)), [0] * int(rng.integers(1, 5))) for _ in range(int(rng.integers(1, 4)))]
+    groups = [(p, [p + int(rng.integers(1, 3 * bs)) for _ in m]) for p, m in groups]
+    singles = [int(rng.integers(2, 4 * bs)) for _ in range(int(rng.integers(0, 4)))]
+    wl = W.shared_prefix_case(seed, groups=groups, singles=singles, num_kv_heads=1, group=1, head_dim=64,
+                              block_size=bs, dtype=W.FP32)
+    geo = wl.geometry
+    a = P.BlockManager(geo.num_blocks, geo.block_size, wl.initial_free_order)
+    b = oracle.BlockManager(geo.num_blocks, geo.block_size, wl.initial_free_order)
+    for op in wl.ops:
+        for m in (a, b):
+            if op.kind == "add":
+                m.add_seq(op.seq, op.n)
+            elif op.kind == "fork":
+                m.fork(op.parent, op.seq, op.n)
+            elif op.kind == "append":
+                m.append_tokens(op.seq, op.n)
+    for k in (1, 2, 3):
+        sa, ga = a.cascade_groups(wl.batch_seqs, k)
+        sb, gb = b.cascade_groups(wl.batch_seqs, k)
+        assert list(sa) == sb and [tuple(g) for g in ga.tolist()] == gb
+
+
+def test_cascade_validation():
+    args = dict(q=FAKE, k_cache=FAKE, v_cache=FAKE, block_tables=FAKE, max_blocks_per_seq=128, context_lens=FAKE,
+                query_start_loc=FAKE, num_seqs=4, num_q_heads=32, max_context_len=2048, shared_blocks=FAKE,
+                groups=FAKE, num_groups=1, max_group_size=4, max_shared_blocks=8, scale=0.088, cache=DESC,
+                out=FAKE, workspace=None, workspace_bytes=0, stream=0)
+    def call(**kw):
+        x = dict(args)
+        x.update(kw)
+        return P.pa_attention_cascade(**x)
+    with pytest.raises(P.PAError) as e:
+        call(cache=(64, 16, 8, 128, P.PA_FP32))
+    assert e.value.status == P.PA_ERR_UNSUPPORTED
+    with pytest.raises(P.PAError):
+        call(num_groups=5)                                      # more groups than sequences
+    with pytest.raises(P.PAError):
+        call(groups=None)
+    with pytest.raises(P.PAError):
+        call(max_shared_blocks=129)                             # beyond the table width
+    with pytest.raises(P.PAError) as e:
+        call()                                                  # no workspace
+    assert "workspace" in str(e.value)
+    need = P.pa_attention_cascade_workspace_size(4, 32, 2048, 8, DESC)
+    assert need > P.pa_attention_workspace_size(4, 32, 1, 2048, DESC)
+    call(num_seqs=0)                                            # empty batch: no-op

@@ -355,3 +355,48 @@ def test_compaction_order_is_ascending_movers_to_ascending_holes():
     assert bm.compact() == [(3, 0), (5, 1), (7, 2)]
     assert bm.blocks_of(0) == [2, 1] and bm.blocks_of(1) == [0]
     assert list(bm.free) == [3, 4, 5, 6, 7]
+
+
+# --------------------------------------------------------------------------
+# cascade groups ([C] §"二、KV Cache管理：从浪费到极致复用": shared prefix pages)
+# --------------------------------------------------------------------------
+
+def _replay_bm(wl):
+    geo = wl.geometry
+    bm = BlockManager(geo.num_blocks, geo.block_size, wl.initial_free_order)
+    for op in wl.ops:
+        if op.kind == "add":
+            bm.add_seq(op.seq, op.n)
+        elif op.kind == "fork":
+            bm.fork(op.parent, op.seq, op.n)
+        elif op.kind == "append":
+            bm.append_tokens(op.seq, op.n)
+    return bm
+
+
+def test_cascade_groups_hand_case():
+    # group 0: 64-token prefix = 4 full blocks of 16, members of 70, 100, 65 tokens;
+    # group 1: 37-token prefix = 2 full blocks (its third block is copied on write);
+    # unshared sequences of 5, 90, 17 tokens sit before each group and at the end
+    wl = W.shared_prefix_case(3, groups=[(64, [70, 100, 65]), (37, [40, 41])], singles=[5, 90, 17],
+                              num_kv_heads=2, group=4, head_dim=128, block_size=16, dtype=W.BF16)
+    bm = _replay_bm(wl)
+    shared, groups = bm.cascade_groups(wl.batch_seqs)
+    assert groups == [(1, 3), (5, 2)]
+    assert shared == [0, 4, 4, 4, 0, 2, 2, 0]
+    # a stricter threshold keeps only the 4-block group
+    shared, groups = bm.cascade_groups(wl.batch_seqs, min_shared_blocks=3)
+    assert groups == [(1, 3)] and shared == [0, 4, 4, 4, 0, 0, 0, 0]
+
+
+def test_cascade_groups_prefix_config():
+    """The shared-prompt configuration: 48 sequences share 124 full blocks
+    (1992 tokens = 124 * 16 + 8; the partly filled 125th block is copied on
+    each sharer's first write)."""
+    wl = W.prefix_cow_decode()
+    bm = _replay_bm(wl)
+    shared, groups = bm.cascade_groups(wl.batch_seqs)
+    assert groups == [(0, 48)]
+    assert shared == [124] * 48 + [0] * 16
+    lead = bm.blocks_of(0)[:124]
+    assert all(bm.blocks_of(s)[:124] == lead for s in range(48))
