@@ -50,10 +50,11 @@ struct PrefillCfg {
   static constexpr int kStageOff = kQBytes;
   static constexpr int kPOff = kStageOff + kNST * kStageBytes;
   static constexpr int kBarOff = kPOff + (kPInK ? 0 : kPBytes);
-  static constexpr int kTmemOff = kBarOff + 8 * 8;
+  static constexpr int kTmemOff = kBarOff + 16 * 8;
   static constexpr int kScanOff = kTmemOff + 16;
   static constexpr int kSeqOff = kScanOff + 32 * 4;
-  static constexpr uint32_t kTmemCols = (kBN + D) <= 128 ? 128 : 256;
+  // S of two tiles (tile j+1's scores are computed during tile j's softmax), then O
+  static constexpr uint32_t kTmemCols = (2 * kBN + D) <= 128 ? 128 : 256;
   static constexpr int kBlocksPerTile = kBN / BS;
   static constexpr uint32_t kIdescS = tc::idesc_bf16_f32(128, kBN, 0, 0);
   static constexpr uint32_t kIdescO = tc::idesc_bf16_f32(128, D, 0, 1);
@@ -103,8 +104,8 @@ __global__ void __launch_bounds__(160, 2)
   uint64_t* q_empty = bars + 1;
   uint64_t* kv_full = bars + 2;   // [2]
   uint64_t* kv_empty = bars + 4;  // [2]
-  uint64_t* s_done = bars + 6;
-  uint64_t* o_done = bars + 7;
+  uint64_t* s_done = bars + 6;    // [2]: S of even / odd tiles
+  uint64_t* o_done = bars + 8;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + C::kTmemOff);
   int* warp_tot = reinterpret_cast<int*>(smem + C::kScanOff);
   int* prefix = reinterpret_cast<int*>(smem + C::kSeqOff);
@@ -122,7 +123,8 @@ __global__ void __launch_bounds__(160, 2)
       mbar_init(&kv_full[i], 1);
       mbar_init(&kv_empty[i], 1);
     }
-    mbar_init(s_done, 1);
+    mbar_init(&s_done[0], 1);
+    mbar_init(&s_done[1], 1);
     mbar_init(o_done, 1);
     fence_barrier_init();
   }
@@ -279,9 +281,24 @@ __global__ void __launch_bounds__(160, 2)
   // ================= warps 0-3: one query row per thread (TMEM lane = row)
   const int r = tid;
   const uint32_t t_lane = tmem + (static_cast<uint32_t>(warp * 32) << 16);
-  const uint32_t s_col = 0, o_col = kBN;
+  const uint32_t o_col = 2 * kBN;
   const uint32_t q_addr = smem_u32(q_s);
   uint32_t it_no = 0, gj = 0;
+  // thread 0: S of global tile g = Q K(g)^T into S buffer g & 1, once K(g) has landed
+  auto issue_s = [&](uint32_t g) {
+    const uint32_t sg = g & 1;
+    mbar_wait(&kv_full[sg], (g >> 1) & 1, a.status);
+    tc::fence_after_sync();
+    const uint32_t k_addr = smem_u32(smem + C::kStageOff + sg * C::kStageBytes);
+#pragma unroll
+    for (int kk = 0; kk < D / 16; ++kk) {
+      const uint32_t off_q = (kk >> 2) * (128 * 128) + (kk & 3) * 32;
+      const uint32_t off_k = (kk >> 2) * (kBN * 128) + (kk & 3) * 32;
+      tc::mma_bf16(tmem + sg * kBN, tc::sw128_desc(q_addr + off_q, 16, 1024), tc::sw128_desc(k_addr + off_k, 16, 1024),
+                   C::kIdescS, kk > 0);
+    }
+    tc::commit(&s_done[sg]);
+  };
   for (int w = blockIdx.x; w < W; w += gridDim.x, ++it_no) {
     Item it = item_of(w);
     finish_item(it);
@@ -290,31 +307,28 @@ __global__ void __launch_bounds__(160, 2)
     const int lim = CASC ? it.L - 1 : min(it.L - it.q_len + tok, it.L - 1);
     float m_used = -CUDART_INF_F, l = 0.f;
     mbar_wait(q_full, it_no & 1, a.status);
+    if (tid == 0) issue_s(gj);
+    __syncwarp();
     for (int j = 0; j < it.ntile; ++j, ++gj) {
       const uint32_t st = gj & 1;
       uint8_t* ks = smem + C::kStageOff + st * C::kStageBytes;
       uint8_t* vs = ks + C::kKBytes;
       uint8_t* ps = C::kPInK ? ks : smem + C::kPOff;
-      if (tid == 0) {
-        mbar_wait(&kv_full[st], (gj >> 1) & 1, a.status);
-        tc::fence_after_sync();
-        const uint32_t k_addr = smem_u32(ks);
-#pragma unroll
-        for (int kk = 0; kk < D / 16; ++kk) {
-          const uint32_t off_q = (kk >> 2) * (128 * 128) + (kk & 3) * 32;
-          const uint32_t off_k = (kk >> 2) * (kBN * 128) + (kk & 3) * 32;
-          tc::mma_bf16(tmem + s_col, tc::sw128_desc(q_addr + off_q, 16, 1024),
-                       tc::sw128_desc(k_addr + off_k, 16, 1024), C::kIdescS, kk > 0);
-        }
-        tc::commit(s_done);
-      }
-      __syncwarp();
-      mbar_wait(s_done, gj & 1, a.status);
+      mbar_wait(&s_done[st], (gj >> 1) & 1, a.status);
       tc::fence_after_sync();
       float sv[kBN];
-      tc::ld32(t_lane + s_col, sv);
-      tc::ld32(t_lane + s_col + 32, sv + 32);
+      tc::ld32(t_lane + st * kBN, sv);
+      tc::ld32(t_lane + st * kBN + 32, sv + 32);
       tc::wait_ld();
+      // The next tile's S goes to the other buffer, whose last reader (this
+      // tile's predecessor) finished before the previous P.V was issued.
+      // Issue it now if its K is already in, so it overlaps this softmax.
+      bool next_issued = false;
+      if (tid == 0 && j + 1 < it.ntile && mbar_test_wait(&kv_full[(gj + 1) & 1], ((gj + 1) >> 1) & 1)) {
+        issue_s(gj + 1);
+        next_issued = true;
+      }
+      __syncwarp();
       const int kbase = j * kBN;
       float mx = -CUDART_INF_F;
 #pragma unroll
@@ -331,8 +345,9 @@ __global__ void __launch_bounds__(160, 2)
         alpha = fast_exp2(m_used - m_new);
         m_used = m_new;
       }
-      // s_done(j) also covers every earlier PV MMA, so O is stable here.
       if (j > 0 && __any_sync(0xffffffffu, bump)) {
+        mbar_wait(o_done, (gj - 1) & 1, a.status);  // O holds every P.V up to tile j-1
+        tc::fence_after_sync();
 #pragma unroll 1
         for (int q = 0; q < D / 32; ++q) {
           float ov[32];
@@ -385,6 +400,7 @@ __global__ void __launch_bounds__(160, 2)
         tc::commit(o_done);
         tc::commit(&kv_empty[st]);
         if (j == it.ntile - 1) tc::commit(q_empty);
+        if (!next_issued && j + 1 < it.ntile) issue_s(gj + 1);
       }
       __syncwarp();
     }
