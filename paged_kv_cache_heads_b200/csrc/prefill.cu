@@ -35,7 +35,7 @@ namespace {
 constexpr int kBN = 64;            // keys per tile
 constexpr float kRescaleLog2 = 8.f;
 
-template <int D, int BS, int GH>
+template <int D, int BS, int GH, int NST>
 struct PrefillCfg {
   static constexpr int kTOK = 128 / GH;          // query tokens per tile
   static constexpr int kHalves = D / 64;         // 128-byte column groups
@@ -45,12 +45,12 @@ struct PrefillCfg {
   static constexpr int kPBytes = 128 * kBN * 2;
   static constexpr bool kPInK = kKBytes >= kPBytes;
   static constexpr int kStageBytes = kKBytes + kVBytes;
-  static constexpr int kNST = 2;
+  static constexpr int kNST = NST;  // K/V stages in the ring
   static constexpr int kQOff = 0;
   static constexpr int kStageOff = kQBytes;
   static constexpr int kPOff = kStageOff + kNST * kStageBytes;
   static constexpr int kBarOff = kPOff + (kPInK ? 0 : kPBytes);
-  static constexpr int kTmemOff = kBarOff + 16 * 8;
+  static constexpr int kTmemOff = kBarOff + ((5 + 2 * NST) * 8 + 15) / 16 * 16;
   static constexpr int kScanOff = kTmemOff + 16;
   static constexpr int kSeqOff = kScanOff + 32 * 4;
   // S of two tiles (tile j+1's scores are computed during tile j's softmax), then O
@@ -91,21 +91,21 @@ struct Item {
   int kb0, chunk;  // cascade prefix pass: first key block of the item's chunk, and its index
 };
 
-template <int D, int BS, int GH, bool CASC>
+template <int D, int BS, int GH, bool CASC, int NST>
 __global__ void __launch_bounds__(160, 2)
     paged_prefill_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constant__ CUtensorMap kmap,
                          const __grid_constant__ CUtensorMap vmap, const PrefillArgs a) {
-  using C = PrefillCfg<D, BS, GH>;
+  using C = PrefillCfg<D, BS, GH, NST>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* q_s = smem + C::kQOff;
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::kBarOff);
   uint64_t* q_full = bars + 0;
   uint64_t* q_empty = bars + 1;
-  uint64_t* kv_full = bars + 2;   // [2]
-  uint64_t* kv_empty = bars + 4;  // [2]
-  uint64_t* s_done = bars + 6;    // [2]: S of even / odd tiles
-  uint64_t* o_done = bars + 8;
+  uint64_t* s_done = bars + 2;    // [2]: S of even / odd tiles
+  uint64_t* o_done = bars + 4;
+  uint64_t* kv_full = bars + 5;   // [NST]
+  uint64_t* kv_empty = kv_full + NST;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + C::kTmemOff);
   int* warp_tot = reinterpret_cast<int*>(smem + C::kScanOff);
   int* prefix = reinterpret_cast<int*>(smem + C::kSeqOff);
@@ -119,7 +119,7 @@ __global__ void __launch_bounds__(160, 2)
   if (tid == 0) {
     mbar_init(q_full, 1);
     mbar_init(q_empty, 1);
-    for (int i = 0; i < 2; ++i) {
+    for (int i = 0; i < NST; ++i) {
       mbar_init(&kv_full[i], 1);
       mbar_init(&kv_empty[i], 1);
     }
@@ -250,8 +250,8 @@ __global__ void __launch_bounds__(160, 2)
         for (int h = 0; h < C::kHalves; ++h)
           tma_load_3d(q_s + h * 128 * 128, &qmap, q_full, h * 64, it.hq0, it.r0 + it.t0);
         for (int j = 0; j < it.ntile; ++j, ++gj) {
-          const uint32_t st = gj & 1;
-          mbar_wait(&kv_empty[st], ((gj >> 1) & 1) ^ 1, a.status);
+          const uint32_t st = gj % NST;
+          mbar_wait(&kv_empty[st], ((gj / NST) & 1) ^ 1, a.status);
           uint8_t* ks = smem + C::kStageOff + st * C::kStageBytes;
           uint8_t* vs = ks + C::kKBytes;
           mbar_arrive_expect_tx(&kv_full[st], C::kStageBytes);
@@ -286,10 +286,10 @@ __global__ void __launch_bounds__(160, 2)
   uint32_t it_no = 0, gj = 0;
   // thread 0: S of global tile g = Q K(g)^T into S buffer g & 1, once K(g) has landed
   auto issue_s = [&](uint32_t g) {
-    const uint32_t sg = g & 1;
-    mbar_wait(&kv_full[sg], (g >> 1) & 1, a.status);
+    const uint32_t sg = g & 1, stg = g % NST;
+    mbar_wait(&kv_full[stg], (g / NST) & 1, a.status);
     tc::fence_after_sync();
-    const uint32_t k_addr = smem_u32(smem + C::kStageOff + sg * C::kStageBytes);
+    const uint32_t k_addr = smem_u32(smem + C::kStageOff + stg * C::kStageBytes);
 #pragma unroll
     for (int kk = 0; kk < D / 16; ++kk) {
       const uint32_t off_q = (kk >> 2) * (128 * 128) + (kk & 3) * 32;
@@ -310,21 +310,21 @@ __global__ void __launch_bounds__(160, 2)
     if (tid == 0) issue_s(gj);
     __syncwarp();
     for (int j = 0; j < it.ntile; ++j, ++gj) {
-      const uint32_t st = gj & 1;
+      const uint32_t st = gj % NST, sb = gj & 1;  // K/V stage, S buffer
       uint8_t* ks = smem + C::kStageOff + st * C::kStageBytes;
       uint8_t* vs = ks + C::kKBytes;
       uint8_t* ps = C::kPInK ? ks : smem + C::kPOff;
-      mbar_wait(&s_done[st], (gj >> 1) & 1, a.status);
+      mbar_wait(&s_done[sb], (gj >> 1) & 1, a.status);
       tc::fence_after_sync();
       float sv[kBN];
-      tc::ld32(t_lane + st * kBN, sv);
-      tc::ld32(t_lane + st * kBN + 32, sv + 32);
+      tc::ld32(t_lane + sb * kBN, sv);
+      tc::ld32(t_lane + sb * kBN + 32, sv + 32);
       tc::wait_ld();
       // The next tile's S goes to the other buffer, whose last reader (this
       // tile's predecessor) finished before the previous P.V was issued.
       // Issue it now if its K is already in, so it overlaps this softmax.
       bool next_issued = false;
-      if (tid == 0 && j + 1 < it.ntile && mbar_test_wait(&kv_full[(gj + 1) & 1], ((gj + 1) >> 1) & 1)) {
+      if (tid == 0 && j + 1 < it.ntile && mbar_test_wait(&kv_full[(gj + 1) % NST], ((gj + 1) / NST) & 1)) {
         issue_s(gj + 1);
         next_issued = true;
       }
@@ -377,7 +377,7 @@ __global__ void __launch_bounds__(160, 2)
       // zero V rows at or beyond L (stale tail of the last block)
       const int vz0 = it.L - kbase;
       if (vz0 < kBN) {
-        mbar_wait(&kv_full[st], (gj >> 1) & 1, a.status);
+        mbar_wait(&kv_full[st], (gj / NST) & 1, a.status);
         const int z0 = vz0 > 0 ? vz0 : 0;
         const int nchunks = (kBN - z0) * C::kHalves * 8;
         for (int i = tid; i < nchunks; i += 128) {
@@ -449,11 +449,11 @@ __global__ void __launch_bounds__(160, 2)
   if (tid == 0) grid_dependency_wait();  // finish no earlier than the previous grid
 }
 
-template <int D, int BS, int GH, bool CASC>
+template <int D, int BS, int GH, bool CASC, int NST>
 cudaError_t launch_prefill_t(const PrefillArgs& a, const CUtensorMap& qmap, const CUtensorMap& kmap,
                              const CUtensorMap& vmap, cudaStream_t stream) {
-  using C = PrefillCfg<D, BS, GH>;
-  auto kern = paged_prefill_kernel<D, BS, GH, CASC>;
+  using C = PrefillCfg<D, BS, GH, NST>;
+  auto kern = paged_prefill_kernel<D, BS, GH, CASC, NST>;
   const size_t smem = C::smem_bytes(a.num_seqs);
   static int configured_smem[64] = {0};
   int dev = 0;
@@ -485,15 +485,27 @@ cudaError_t launch_prefill_t(const PrefillArgs& a, const CUtensorMap& qmap, cons
   return launch_chained(kern, dim3(grid), dim3(160), smem, stream, qmap, kmap, vmap, a);
 }
 
+// K/V ring depth. Two 32 KiB stages keep the CTA at ~100 KB of shared memory,
+// so two CTAs share an SM and overlap each other's softmax and MMA chains;
+// five stages at one CTA per SM measured slower (82.6 vs 66.6 us on the
+// mixed batch's prefill rows).
+constexpr int kPrefillStages = 2;
+
+template <int D, int BS, int GH, bool CASC>
+cudaError_t launch_prefill_st(const PrefillArgs& a, const CUtensorMap& qmap, const CUtensorMap& kmap,
+                              const CUtensorMap& vmap, cudaStream_t stream) {
+  return launch_prefill_t<D, BS, GH, CASC, kPrefillStages>(a, qmap, kmap, vmap, stream);
+}
+
 template <int D, int BS, bool CASC>
 cudaError_t launch_prefill_gh(const PrefillArgs& a, const CUtensorMap& qmap, const CUtensorMap& kmap,
                               const CUtensorMap& vmap, int gh, cudaStream_t stream) {
   switch (gh) {
-    case 16: return launch_prefill_t<D, BS, 16, CASC>(a, qmap, kmap, vmap, stream);
-    case 8: return launch_prefill_t<D, BS, 8, CASC>(a, qmap, kmap, vmap, stream);
-    case 4: return launch_prefill_t<D, BS, 4, CASC>(a, qmap, kmap, vmap, stream);
-    case 2: return launch_prefill_t<D, BS, 2, CASC>(a, qmap, kmap, vmap, stream);
-    default: return launch_prefill_t<D, BS, 1, CASC>(a, qmap, kmap, vmap, stream);
+    case 16: return launch_prefill_st<D, BS, 16, CASC>(a, qmap, kmap, vmap, stream);
+    case 8: return launch_prefill_st<D, BS, 8, CASC>(a, qmap, kmap, vmap, stream);
+    case 4: return launch_prefill_st<D, BS, 4, CASC>(a, qmap, kmap, vmap, stream);
+    case 2: return launch_prefill_st<D, BS, 2, CASC>(a, qmap, kmap, vmap, stream);
+    default: return launch_prefill_st<D, BS, 1, CASC>(a, qmap, kmap, vmap, stream);
   }
 }
 
