@@ -46,11 +46,22 @@ NCU_TRAFFIC = {}
 
 
 def _sources_digest() -> str:
+    """Digest of every kernel source: recorded ncu traffic is used only while it matches."""
     h = hashlib.sha256()
-    for f in ("decode.cu", "prefill.cu", "pa_common.cuh"):
-        with open(os.path.join(ROOT, "paged_kv_cache_heads_b200", "csrc", f), "rb") as fh:
-            h.update(fh.read())
+    csrc = os.path.join(ROOT, "paged_kv_cache_heads_b200", "csrc")
+    for f in sorted(os.listdir(csrc)):
+        if f.endswith((".cu", ".cuh", ".h")):
+            with open(os.path.join(csrc, f), "rb") as fh:
+                h.update(f.encode() + fh.read())
     return h.hexdigest()[:16]
+
+
+def decode_kernel_name(geo) -> str:
+    """The decode kernel libpa picks for this geometry (its policy for a plain
+    pa_attention call: tensor cores for bf16, head_dim 128, groups of 2/4/8)."""
+    env = os.environ.get("PA_DECODE_TC", "")
+    tc = geo.dtype == "bf16" and geo.head_dim == 128 and geo.group in (2, 4, 8) and env != "0"
+    return "paged_decode_tc_kernel" if tc else "paged_decode_kernel"
 
 
 def measured_peaks():
@@ -574,8 +585,8 @@ def main():
         dist.destroy_process_group()
     if rank != 0:
         return 0
-    roof = {"kernel": "pa_attention (paged_decode_kernel + decode_combine_kernel%s)"
-                      % (" + paged_prefill_kernel" if wl.max_query_len > 1 else ""),
+    roof = {"kernel": "pa_attention (%s + decode_combine_kernel%s)"
+                      % (decode_kernel_name(wl.geometry), " + paged_prefill_kernel" if wl.max_query_len > 1 else ""),
             "bound": "hbm", "achieved": achieved, "peak": hbm_peak, "unit": "GB/s",
             "frac": achieved / hbm_peak, "traffic": traffic, "peak_source": peak_src + " (MEASURED_PEAKS.json hbm_gbs)"
             if peak_src == "measured" else "fallback 6.65 TB/s",

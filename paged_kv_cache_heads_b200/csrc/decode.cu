@@ -559,6 +559,7 @@ cudaError_t launch_decode_t(DecodeArgs& a, const CUtensorMap& kmap, const CUtens
     if (v >= 1 && v < grid) grid = v;
   }
   a.grid = grid;
+  a.hpu = C::kHPU;
   log_launch("paged_decode_kernel", grid, C::kThreads, smem, per_sm);
   return launch_chained(kern, dim3(grid), dim3(C::kThreads), smem, stream, kmap, vmap, a);
 }
@@ -595,7 +596,8 @@ cudaError_t launch_combine_t(const DecodeArgs& a, cudaStream_t stream) {
 
 template <typename T, int D, int BS>
 cudaError_t launch_combine_gh(const DecodeArgs& a, const pa_cache_desc& desc, cudaStream_t stream) {
-  switch (decode_heads_per_unit(a.num_q_heads / a.num_kv_heads, desc)) {
+  (void)desc;
+  switch (a.hpu) {  // the unit of the decode grid that was launched
     case 8: return launch_combine_t<T, D, BS, 8>(a, stream);
     case 4: return launch_combine_t<T, D, BS, 4>(a, stream);
     case 2: return launch_combine_t<T, D, BS, 2>(a, stream);
@@ -628,7 +630,6 @@ int32_t decode_kv_heads_per_cta(int32_t group, const pa_cache_desc& c) {
 }
 
 int32_t decode_heads_per_unit(int32_t group, const pa_cache_desc& c) {
-  if (decode_uses_tc(group, c)) return group;  // one unit per KV head
   return decode_heads_per_cta(group) * decode_kv_heads_per_cta(group, c);
 }
 

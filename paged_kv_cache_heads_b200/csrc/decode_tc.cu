@@ -543,6 +543,7 @@ cudaError_t launch_tc_t(DecodeArgs& a, const CUtensorMap& qmap, const CUtensorMa
     if (v >= 1 && v < grid) grid = v;
   }
   a.grid = grid;
+  a.hpu = GH;
   log_launch("paged_decode_tc_kernel", grid, C::kThreads, smem, 1);
   return launch_chained(kern, dim3(grid), dim3(C::kThreads), smem, stream, qmap, kmap, vmap, a);
 }
@@ -572,12 +573,17 @@ cudaError_t launch_tc_gh(DecodeArgs& a, const CUtensorMap& qmap, const CUtensorM
 
 }  // namespace
 
-bool decode_uses_tc(int32_t group, const pa_cache_desc& c) {
-  static const bool disabled = [] {
+bool decode_tc_supported(int32_t group, const pa_cache_desc& c) {
+  return c.dtype == PA_BF16 && c.head_dim == 128 && (group == 2 || group == 4 || group == 8);
+}
+
+bool decode_uses_tc(int32_t group, const pa_cache_desc& c, bool short_units) {
+  static const int mode = [] {  // -1: by workload, 0: never, 1: always
     const char* env = getenv("PA_DECODE_TC");
-    return env && env[0] == '0';
+    return env && (env[0] == '0' || env[0] == '1') ? env[0] - '0' : -1;
   }();
-  return !disabled && c.dtype == PA_BF16 && c.head_dim == 128 && (group == 2 || group == 4 || group == 8);
+  if (!decode_tc_supported(group, c) || mode == 0) return false;
+  return mode == 1 || !short_units;
 }
 
 cudaError_t launch_decode_tc(DecodeArgs& a, const CUtensorMap& qmap, const CUtensorMap& kmap,

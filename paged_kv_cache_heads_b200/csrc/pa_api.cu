@@ -1,6 +1,7 @@
 // C ABI of libpa: host-side validation, TMA tensor-map encoding, the device
 // status word, and dispatch to the kernels. See include/pa.h for the contract
 // of every entry point.
+#include <algorithm>
 #include <cuda.h>
 #include <cuda_runtime.h>
 
@@ -280,14 +281,14 @@ namespace {
 // launch status; the return value reports a tensor-map failure.
 pa_status launch_decode_path(DecodeArgs& a, const void* q, const void* k_cache, const void* v_cache,
                              int32_t num_q_heads, int32_t num_q_tokens, const pa_cache_desc* cache,
-                             cudaStream_t s, cudaError_t* e) {
+                             bool short_units, cudaStream_t s, cudaError_t* e) {
   pa_status st;
   const int32_t group = num_q_heads / cache->num_kv_heads;
   // q as a 3-D tensor {head_dim, num_q_heads, num_q_tokens}
   const uint64_t qd[3] = {uint64_t(cache->head_dim), uint64_t(num_q_heads), uint64_t(num_q_tokens)};
   const uint64_t qs[2] = {uint64_t(cache->head_dim) * 2, uint64_t(num_q_heads) * cache->head_dim * 2};
   CUtensorMap kmap, vmap;
-  if (decode_uses_tc(group, *cache)) {
+  if (decode_uses_tc(group, *cache, short_units)) {
     // tensor-core decode: 64-column (128-byte) swizzled boxes, Q^T per KV head
     CUtensorMap qmap;
     const uint32_t qbox[3] = {64, uint32_t(group), 1};
@@ -316,10 +317,15 @@ bool workspace_layout(int32_t num_seqs, int32_t num_q_heads, int32_t max_query_l
     return false;
   *w = WorkspaceLayout();
   if (max_query_len < 1 || num_seqs == 0) return true;
-  const int32_t gh = decode_heads_per_unit(num_q_heads / cache->num_kv_heads, *cache);
-  // partial slot u + c for unit u = (sequence, head group) and covering CTA c
-  const size_t slots = size_t(num_seqs) * (num_q_heads / gh) + size_t(decode_max_grid());
-  const size_t parts = slots * gh;
+  // partial slot u + c for unit u = (sequence, head group) and covering CTA c,
+  // sized for whichever decode kernel the call may choose
+  const int32_t group = num_q_heads / cache->num_kv_heads;
+  size_t parts = 0;
+  for (int32_t gh : {decode_heads_per_unit(group, *cache), decode_tc_supported(group, *cache) ? group : 0}) {
+    if (gh < 1) continue;
+    const size_t slots = size_t(num_seqs) * (num_q_heads / gh) + size_t(decode_max_grid());
+    parts = std::max(parts, slots * gh);
+  }
   w->lse_off = (parts * cache->head_dim * 4 + 255) & ~size_t(255);
   w->prefix_off = (w->lse_off + parts * 4 + 255) & ~size_t(255);
   w->bytes = w->prefix_off + (size_t(num_seqs) + 1) * 4;
@@ -395,6 +401,7 @@ pa_status pa_attention(const void* q, const void* k_cache, const void* v_cache,
   a.num_blocks = cache->num_blocks;
   a.max_context_len = max_context_len;
   a.grid = 0;
+  a.hpu = 1;
   a.scale_log2 = scale_log2;
   a.skip_blocks = nullptr;
   a.l1_o = nullptr;
@@ -405,7 +412,8 @@ pa_status pa_attention(const void* q, const void* k_cache, const void* v_cache,
   const int32_t group = num_q_heads / cache->num_kv_heads;
   const uint64_t qd[3] = {uint64_t(cache->head_dim), uint64_t(num_q_heads), uint64_t(num_q_tokens)};
   const uint64_t qs[2] = {uint64_t(cache->head_dim) * 2, uint64_t(num_q_heads) * cache->head_dim * 2};
-  if ((st = launch_decode_path(a, q, k_cache, v_cache, num_q_heads, num_q_tokens, cache, s, &e)) != PA_OK) return st;
+  if ((st = launch_decode_path(a, q, k_cache, v_cache, num_q_heads, num_q_tokens, cache, false, s, &e)) != PA_OK)
+    return st;
   if (e != cudaSuccess) return cuda_fail(e, "decode launch");
   e = launch_decode_combine(a, *cache, s);
   if (e != cudaSuccess) return cuda_fail(e, "decode combine launch");
@@ -547,6 +555,7 @@ pa_status pa_attention_cascade(const void* q, const void* k_cache, const void* v
   a.num_blocks = cache->num_blocks;
   a.max_context_len = max_context_len;
   a.grid = 0;
+  a.hpu = 1;
   a.scale_log2 = scale_log2;
   a.skip_blocks = num_groups > 0 ? shared_blocks : nullptr;
   a.l1_o = reinterpret_cast<float*>(ws + wl.l1_o_off);
@@ -555,7 +564,10 @@ pa_status pa_attention_cascade(const void* q, const void* k_cache, const void* v
   a.l1_chunk_blocks = chunk_blocks;
 
   // 1. every sequence's own blocks (past its group's shared ones): partials
-  if ((st = launch_decode_path(a, q, k_cache, v_cache, num_q_heads, num_seqs, cache, s, &e)) != PA_OK) return st;
+  // the suffix pass: each sequence's own blocks are typically few
+  if ((st = launch_decode_path(a, q, k_cache, v_cache, num_q_heads, num_seqs, cache, num_groups > 0, s, &e)) !=
+      PA_OK)
+    return st;
   if (e != cudaSuccess) return cuda_fail(e, "decode launch");
   // 2. each group's shared blocks, read once for all its members: partials
   if (num_groups > 0) {

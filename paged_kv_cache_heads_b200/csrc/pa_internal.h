@@ -28,7 +28,8 @@ struct DecodeArgs {
   int32_t num_kv_heads;
   int32_t num_blocks;
   int32_t max_context_len;
-  int32_t grid;         // CTAs of the decode grid (set by launch_decode)
+  int32_t grid;         // CTAs of the decode grid (set by the decode launcher)
+  int32_t hpu;          // query heads per unit of the decode grid (set by the decode launcher)
   float scale_log2;     // scale * log2(e)
   // Cascade (shared-prefix) decode; all null / 0 otherwise.
   const int32_t* skip_blocks;  // [num_seqs] leading table blocks read by the prefix pass instead
@@ -81,11 +82,15 @@ cudaError_t launch_copy_blocks(const int32_t* pairs, int32_t num_pairs, void* k_
                                cudaStream_t stream);
 cudaError_t launch_decode(DecodeArgs& a, const CUtensorMap& kmap, const CUtensorMap& vmap,
                           const pa_cache_desc& c, cudaStream_t stream);
-// Grouped-query decode on the tensor cores: bf16, head_dim 128, group 2, 4 or 8
-// (environment PA_DECODE_TC=0 selects the CUDA-core kernel instead). `qmap` is
-// q as {head_dim, num_q_heads, num_q_tokens} with box {64, group, 1}; the cache
-// maps have box {64, 1, block_size, 1}; all three use the 128-byte swizzle.
-bool decode_uses_tc(int32_t group, const pa_cache_desc& c);
+// Grouped-query decode on the tensor cores: bf16, head_dim 128, group 2, 4 or 8.
+// It wins on long units (128-token tiles); the CUDA-core kernel streams block
+// by block and wins when units are a few blocks long, as in the suffix pass of
+// cascade decode (`short_units`). Environment PA_DECODE_TC=0 never selects the
+// tensor-core kernel, PA_DECODE_TC=1 always does where supported.
+// `qmap` is q as {head_dim, num_q_heads, num_q_tokens} with box {64, group, 1};
+// the cache maps have box {64, 1, block_size, 1}; all three use the 128-byte swizzle.
+bool decode_tc_supported(int32_t group, const pa_cache_desc& c);
+bool decode_uses_tc(int32_t group, const pa_cache_desc& c, bool short_units);
 cudaError_t launch_decode_tc(DecodeArgs& a, const CUtensorMap& qmap, const CUtensorMap& kmap,
                              const CUtensorMap& vmap, const pa_cache_desc& c, cudaStream_t stream);
 cudaError_t launch_decode_combine(const DecodeArgs& a, const pa_cache_desc& c, cudaStream_t stream);
@@ -125,6 +130,7 @@ void log_launch(const char* kernel, int grid, int block, size_t smem, int per_sm
 // KV heads one decode CTA streams together (adjacent heads; only without GQA),
 // and query heads per decode unit (heads per CTA x KV heads per CTA).
 int32_t decode_kv_heads_per_cta(int32_t group, const pa_cache_desc& c);
+// Query heads per unit of the CUDA-core kernel (the tensor-core kernel's unit is the whole group).
 int32_t decode_heads_per_unit(int32_t group, const pa_cache_desc& c);
 // Heads of one GQA group handled together by one decode CTA.
 int32_t decode_heads_per_cta(int32_t group);

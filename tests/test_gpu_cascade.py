@@ -135,3 +135,43 @@ def test_cascade_graph_replay(P):
     torch.cuda.synchronize()
     assert torch.equal(eager, b.out)
     assert P.pa_read_device_flags(clear=True) == 0
+
+
+_FORCED_TC_SCRIPT = r'''
+import sys, numpy as np, torch
+sys.path.insert(0, sys.argv[1])
+from oracle import scenario as oscen
+from paged_kv_cache_heads_b200 import workloads as W, scenario as gs
+import paged_kv_cache_heads_b200 as P
+for seed, g, bs in [(31, 4, 16), (32, 8, 8), (33, 2, 32)]:
+    rng = np.random.default_rng(seed)
+    groups = [(int(rng.integers(300, 700)), [0] * 3), (int(rng.integers(40, 200)), [0] * 37)]
+    groups = [(p, [p + int(rng.integers(1, 300)) for _ in m]) for p, m in groups]
+    wl = W.shared_prefix_case(seed, groups=groups, singles=[17, 700], num_kv_heads=2, group=g, head_dim=128,
+                              block_size=bs, dtype=W.BF16)
+    b = gs.prepare(wl)
+    gs.run_step(b)
+    plan = gs.plan_cascade(b)
+    out = torch.zeros_like(b.out)
+    gs.run_attention_cascade(b, plan, out=out)
+    torch.cuda.synchronize()
+    o = oscen.run(wl, W.sentinel_cache(wl.geometry), W.sentinel_cache(wl.geometry))
+    err = np.abs(gs.out_as_f64(out, W.BF16) - o.out)
+    assert np.isfinite(err).all() and err.max() <= 2e-2 and err.mean() <= 2e-3, (seed, err.max(), err.mean())
+assert P.pa_read_device_flags(clear=True) == 0
+print("OK")
+'''
+
+
+def test_cascade_with_tensor_core_suffix_pass(P):
+    """The suffix pass runs on the CUDA-core kernel by default (short units);
+    PA_DECODE_TC=1 forces the tensor-core kernel, whose skipping of shared
+    blocks must give the same results."""
+    import os
+    import subprocess
+    import sys
+    root = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+    env = dict(os.environ, PA_DECODE_TC="1")
+    r = subprocess.run([sys.executable, "-c", _FORCED_TC_SCRIPT, root], capture_output=True, text=True, env=env,
+                       cwd=root, timeout=600)
+    assert r.returncode == 0 and "OK" in r.stdout, r.stdout + r.stderr
