@@ -42,7 +42,13 @@ UNIT = "query-tokens/s"
 # DRAM bytes per attention call from one ncu capture of this workload
 # (dram__bytes_read.sum + dram__bytes_write.sum, both attention kernels),
 # valid only while the kernel sources are byte-identical to the captured ones.
-NCU_TRAFFIC = {}
+# DRAM bytes (read + write) of one launch of the workload's decode kernel, from
+# `ncu --set full` captures (profiles/), valid while the kernel sources match.
+NCU_TRAFFIC = {
+    "sources": "dabaf38d1493154f",
+    "llama7b_decode_b32_bf16": 589814784 + 5732096,    # paged_decode_kernel
+    "gqa_long_decode_b16_bf16": 166983424 + 3899136,   # paged_decode_tc_kernel
+}
 
 
 def _sources_digest() -> str:
