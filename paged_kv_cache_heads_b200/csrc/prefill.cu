@@ -330,12 +330,29 @@ __global__ void __launch_bounds__(160, 2)
       }
       __syncwarp();
       const int kbase = j * kBN;
+      // With a positive scale the row max is taken on the raw scores and the
+      // scale is folded into the exponent's FMA below; the causal mask is
+      // applied only on tiles that reach past this row's last visible key.
+      float sc = a.scale_log2;
       float mx = -CUDART_INF_F;
+      if (sc > 0.f && kbase + kBN - 1 <= lim) {
 #pragma unroll
-      for (int c = 0; c < kBN; ++c) {
-        sv[c] = (kbase + c <= lim) ? sv[c] * a.scale_log2 : -CUDART_INF_F;
-        mx = fmaxf(mx, sv[c]);
+        for (int c = 0; c < kBN; ++c) mx = fmaxf(mx, sv[c]);
+      } else if (sc > 0.f) {
+#pragma unroll
+        for (int c = 0; c < kBN; ++c) {
+          if (kbase + c > lim) sv[c] = -CUDART_INF_F;
+          mx = fmaxf(mx, sv[c]);
+        }
+      } else {
+#pragma unroll
+        for (int c = 0; c < kBN; ++c) {
+          sv[c] = (kbase + c <= lim) ? sv[c] * sc : -CUDART_INF_F;
+          mx = fmaxf(mx, sv[c]);
+        }
+        sc = 1.f;  // already scaled
       }
+      mx *= sc;
       // Rescale only when the running max grows by more than 2^8; otherwise
       // keep the old reference so P stays below 2^8 and O needs no update.
       const float m_new = fmaxf(m_used, mx);
@@ -366,8 +383,8 @@ __global__ void __launch_bounds__(160, 2)
         uint32_t pk[4];
 #pragma unroll
         for (int i = 0; i < 4; ++i) {
-          const float p0 = fast_exp2(sv[c8 * 8 + 2 * i] - m_used);
-          const float p1 = fast_exp2(sv[c8 * 8 + 2 * i + 1] - m_used);
+          const float p0 = fast_exp2(fmaf(sv[c8 * 8 + 2 * i], sc, -m_used));
+          const float p1 = fast_exp2(fmaf(sv[c8 * 8 + 2 * i + 1], sc, -m_used));
           l += p0 + p1;
           const __nv_bfloat162 h2 = __floats2bfloat162_rn(p0, p1);
           pk[i] = *reinterpret_cast<const uint32_t*>(&h2);
