@@ -45,20 +45,26 @@ UNIT = "query-tokens/s"
 # DRAM bytes (read + write) of one launch of the workload's decode kernel, from
 # `ncu --set full` captures (profiles/), valid while the kernel sources match.
 NCU_TRAFFIC = {
-    "sources": "dabaf38d1493154f",
+    "sources": "2206ee5dbfc757b4",   # decode kernel sources of the capture
     "llama7b_decode_b32_bf16": 589814784 + 5732096,    # paged_decode_kernel
     "gqa_long_decode_b16_bf16": 166983424 + 3899136,   # paged_decode_tc_kernel
 }
 
 
+# Every source the decode kernels are compiled from: recorded ncu traffic of a
+# decode kernel is used only while these files are unchanged.
+DECODE_SOURCES = ("decode.cu", "decode_tc.cu", "decode_common.cuh", "pa_common.cuh", "pa_internal.h",
+                  "tcgen05.cuh")
+
+
 def _sources_digest() -> str:
-    """Digest of every kernel source: recorded ncu traffic is used only while it matches."""
     h = hashlib.sha256()
     csrc = os.path.join(ROOT, "paged_kv_cache_heads_b200", "csrc")
-    for f in sorted(os.listdir(csrc)):
-        if f.endswith((".cu", ".cuh", ".h")):
-            with open(os.path.join(csrc, f), "rb") as fh:
-                h.update(f.encode() + fh.read())
+    for f in DECODE_SOURCES:
+        with open(os.path.join(csrc, f), "rb") as fh:
+            h.update(f.encode() + fh.read())
+    with open(os.path.join(ROOT, "include", "pa.h"), "rb") as fh:
+        h.update(fh.read())
     return h.hexdigest()[:16]
 
 
@@ -340,19 +346,16 @@ def measure_ours(wl, steps: int, warmup: int, device, gpu_index: int):
     if ms_graph <= ms_eager:
         clocks = clocks_g
 
-    # ---- end to end: inputs from pinned host memory, output read back, same calls
-    host_in = [t.cpu().pin_memory() for t in (b.q, b.step_k, b.step_v, b.step_slots, b.step_pairs,
-                                              b.block_tables, b.context_lens, b.query_start_loc)]
-    dev_in = [b.q, b.step_k, b.step_v, b.step_slots, b.step_pairs, b.block_tables, b.context_lens,
-              b.query_start_loc]
+    # ---- end to end: every step's inputs (q, new K/V rows, slots, CoW pairs,
+    # tables, lengths, query starts) staged in one pinned host buffer and sent
+    # with one copy; the output read back; the same library calls in between
+    host_in, dev_in = gs.pack_step_inputs(b)
     host_out = torch.empty(b.out.shape, dtype=b.out.dtype).pin_memory()
-    h2d = sum(t.numel() * t.element_size() for t in host_in)
+    h2d = host_in.numel() * host_in.element_size()
     d2h = host_out.numel() * host_out.element_size()
 
     def e2e_step():
-        for h, d in zip(host_in, dev_in):
-            if h.numel():
-                d.copy_(h, non_blocking=True)
+        dev_in.copy_(host_in, non_blocking=True)
         gs.run_step(b)
         host_out.copy_(b.out, non_blocking=True)
 
@@ -371,9 +374,7 @@ def measure_ours(wl, steps: int, warmup: int, device, gpu_index: int):
 
     # ---- the same e2e step captured once in a CUDA graph (copies in, step, copy out)
     def pre():
-        for h, d in zip(host_in, dev_in):
-            if h.numel():
-                d.copy_(h, non_blocking=True)
+        dev_in.copy_(host_in, non_blocking=True)
 
     graph = gs.capture_step(b, pre=pre, post=lambda: host_out.copy_(b.out, non_blocking=True))
     for _ in range(max(warmup, 1)):

@@ -212,3 +212,33 @@ def run_attention_cascade(b: DeviceBatch, plan: CascadePlan, stream=None, out=No
                          plan.shared_blocks, plan.groups, plan.num_groups, plan.max_group_size,
                          plan.max_shared_blocks, b.wl.scale, b.desc, b.out if out is None else out,
                          plan.workspace, stream=stream)
+
+
+STEP_INPUTS = ("q", "step_k", "step_v", "step_slots", "step_pairs", "block_tables", "context_lens",
+               "query_start_loc")
+
+
+def pack_step_inputs(b: DeviceBatch):
+    """Stage every per-step input in one buffer so that it arrives with a single copy.
+
+    Returns ``(host, dev)``: a pinned host buffer and a device buffer with the
+    same layout (each input at a 256-byte aligned offset). The batch's input
+    tensors become views of ``dev``, so the library reads them in place; a
+    serving loop writes the next step's inputs into ``host`` and issues one
+    ``dev.copy_(host, non_blocking=True)``.
+    """
+    layout, total = [], 0
+    for name in STEP_INPUTS:
+        t = getattr(b, name)
+        nbytes = t.numel() * t.element_size()
+        layout.append((name, total, nbytes))
+        total += (nbytes + 255) // 256 * 256
+    dev = torch.empty(max(total, 256), dtype=torch.uint8, device=b.q.device)
+    host = torch.empty(max(total, 256), dtype=torch.uint8).pin_memory()
+    for name, off, nbytes in layout:
+        t = getattr(b, name)
+        view = dev[off:off + nbytes].view(t.dtype).view(t.shape)
+        view.copy_(t)
+        host[off:off + nbytes].copy_(t.detach().cpu().contiguous().view(-1).view(torch.uint8))
+        setattr(b, name, view)
+    return host, dev

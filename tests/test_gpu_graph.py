@@ -66,3 +66,22 @@ def test_graph_with_host_copies(torch_cuda):
     graph.replay()
     torch.cuda.synchronize()
     assert torch.equal(out_host, want)
+
+
+def test_packed_step_inputs_one_copy(torch_cuda):
+    """All of a step's inputs staged in one pinned buffer: one host-to-device
+    copy, then the usual calls, give the eager result bit for bit."""
+    torch = torch_cuda
+    from paged_kv_cache_heads_b200 import scenario as gs
+    wl = W.CONFIGS["mixed_bs8"]()
+    b = gs.prepare(wl)
+    gs.run_step(b)
+    torch.cuda.synchronize()
+    want = b.out.clone()
+    host, dev = gs.pack_step_inputs(b)
+    dev.zero_()                                  # nothing left on the device but the caches
+    b.out.zero_()
+    dev.copy_(host, non_blocking=True)
+    gs.run_step(b)
+    torch.cuda.synchronize()
+    assert torch.equal(b.out, want)
