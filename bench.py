@@ -45,9 +45,9 @@ UNIT = "query-tokens/s"
 # DRAM bytes (read + write) of one launch of the workload's decode kernel, from
 # `ncu --set full` captures (profiles/), valid while the kernel sources match.
 NCU_TRAFFIC = {
-    "sources": "2206ee5dbfc757b4",   # decode kernel sources of the capture
-    "llama7b_decode_b32_bf16": 589814784 + 5732096,    # paged_decode_kernel
-    "gqa_long_decode_b16_bf16": 166983424 + 3899136,   # paged_decode_tc_kernel
+    "sources": "14d3d4a5902253c7",   # decode kernel sources of the capture
+    "llama7b_decode_b32_bf16": 589815040 + 4682240,    # paged_decode_kernel
+    "gqa_long_decode_b16_bf16": 166957824 + 3845120,   # paged_decode_tc_kernel
 }
 
 

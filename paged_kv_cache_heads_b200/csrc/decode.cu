@@ -12,6 +12,10 @@
 // bandwidth (§"三、连续批处理：让GPU一刻不停" of the first page), which shapes
 // the design.
 //
+// This CUDA-core kernel serves fp32 caches, head_dim 64, ungrouped heads and
+// the suffix pass of cascade decode (short units); grouped bf16 heads of 128
+// run on the tensor cores (decode_tc.cu), with the same partition and merge.
+//
 // Design (B200):
 //  * A unit is (sequence, group of GH query heads sharing one KV head); its
 //    work is the sequence's ceil(L/bs) KV blocks of that head. All units'
@@ -29,6 +33,11 @@
 //    head's exp, and the lanes exchange probabilities for P.V. Warps merge
 //    their (m, l, acc) through shared memory at the end of a segment.
 //  * GQA: every KV block is read once for the GH query heads of its group.
+//    Without grouping and with Hkv a multiple of 4, a unit is 4 adjacent KV
+//    heads: one box {D, 4, bs, 1} reads 4*D contiguous elements per token and
+//    consumer warp w owns head w of every block.
+//  * Cascade decode: a sequence's first skip_blocks[s] blocks are left to the
+//    prefix pass; its units stream the rest and always leave a partial.
 //  * Keys at or beyond L (the unfilled tail of the last block) are masked and
 //    their V rows are never read, so stale bits there (even NaN) cannot leak.
 //  * A unit covered by one CTA writes its output rows directly. Otherwise each
@@ -443,14 +452,13 @@ __global__ void __launch_bounds__((NCW + 1) * 32, (GH == 1 ? 4 : 3))
 
 // One CTA per unit (sequence, head group), GH x D threads: merge the
 // partials of a unit that several CTAs streamed and, for a cascade sequence,
-// the prefix-pass partials of its shared blocks. The weights
-// 2^(lse_j - M) / sum are formed in parallel in shared memory, then each
-// thread sums its (head, column) over the partials.
+// the prefix-pass partials of its shared blocks, with weights
+// 2^(lse_j - M) / sum_j 2^(lse_j - M). Each thread merges its own (head,
+// column) with a running max, so no shared memory and no block barrier.
 template <typename T, int D, int BS, int GH>  // GH here: query heads per unit
 __global__ void __launch_bounds__(GH * D) decode_combine_kernel(const DecodeArgs a) {
   launch_dependents();
   grid_dependency_wait();  // the decode grid (partials and the block prefix) is complete
-  extern __shared__ float wsm[];  // [n][GH] weights, then [GH] max and [GH] sum
   const int HG = a.num_q_heads / GH;
   const int u = blockIdx.x;
   const int s = u / HG, hg = u - s * HG;
@@ -467,66 +475,50 @@ __global__ void __launch_bounds__(GH * D) decode_combine_kernel(const DecodeArgs
     if (n2 == 1 && n1 == 0) return;  // one CTA covered the unit and wrote its rows
   }
   const int n = n2 + n1;
-  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-  float* mx = wsm + n * GH;
-  float* sm = mx + GH;
+  const int tid = threadIdx.x;
+  const int gi = tid / D, d = tid - gi * D;  // this thread's (head, column)
   const size_t slot0 = static_cast<size_t>(u) + c0;
-  const size_t l1_row = static_cast<size_t>(s) * a.num_q_heads + static_cast<size_t>(hg) * GH;  // + gi
+  const size_t l1_row = (static_cast<size_t>(s) * a.num_q_heads + static_cast<size_t>(hg) * GH + gi) * a.l1_max_chunks;
+  const int64_t Bt = static_cast<int64_t>(a.seq_prefix[a.num_seqs]) * HG;
   // With more CTAs than blocks some CTAs in [c0, c0 + n2) stream nothing and
-  // wrote no partial: they get weight 0 (and their slot is never read).
+  // wrote no partial: they get weight 0 (and their stale slot is never read).
   auto streams = [&](int cc) {
-    return static_cast<int64_t>(cc) * (static_cast<int64_t>(a.seq_prefix[a.num_seqs]) * HG) / a.grid <
-           static_cast<int64_t>(cc + 1) * (static_cast<int64_t>(a.seq_prefix[a.num_seqs]) * HG) / a.grid;
+    return static_cast<int64_t>(cc) * Bt / a.grid < static_cast<int64_t>(cc + 1) * Bt / a.grid;
   };
-  for (int i = tid; i < n * GH; i += blockDim.x) {
-    const int j = i / GH, gi = i - j * GH;
-    if (j < n2)
-      wsm[i] = streams(c0 + j) ? a.part_lse[(slot0 + j) * GH + gi] : -CUDART_INF_F;
-    else
-      wsm[i] = a.l1_lse[(l1_row + gi) * a.l1_max_chunks + (j - n2)];
-  }
-  __syncthreads();
-  if (warp < GH) {  // warp g reduces head g over the n partials
-    float m = -CUDART_INF_F;
-    for (int j = lane; j < n; j += 32) m = fmaxf(m, wsm[j * GH + warp]);
+  // Each thread folds its partials with a running max (weights 2^(lse - M));
+  // loads are issued four at a time, ahead of the arithmetic.
+  float M = -CUDART_INF_F, sum = 0.f, acc = 0.f;
+  for (int j0 = 0; j0 < n; j0 += 4) {
+    float lse[4], val[4];
 #pragma unroll
-    for (int off = 16; off > 0; off >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, off));
-    float t = 0.f;
-    for (int j = lane; j < n; j += 32) t += fast_exp2(wsm[j * GH + warp] - m);
+    for (int q = 0; q < 4; ++q) {
+      const int j = j0 + q;
+      lse[q] = -CUDART_INF_F;
+      val[q] = 0.f;
+      if (j < n2) {
+        if (streams(c0 + j)) {
+          const size_t part = (slot0 + j) * GH + gi;
+          lse[q] = a.part_lse[part];
+          val[q] = a.part_o[part * D + d];
+        }
+      } else if (j < n) {
+        lse[q] = a.l1_lse[l1_row + (j - n2)];
+        val[q] = a.l1_o[(l1_row + (j - n2)) * D + d];
+      }
+    }
 #pragma unroll
-    for (int off = 16; off > 0; off >>= 1) t += __shfl_xor_sync(0xffffffffu, t, off);
-    if (lane == 0) {
-      mx[warp] = m;
-      sm[warp] = t;
+    for (int q = 0; q < 4; ++q) {
+      if (lse[q] == -CUDART_INF_F) continue;
+      const float m_new = fmaxf(M, lse[q]);
+      const float keep = fast_exp2(M - m_new), w = fast_exp2(lse[q] - m_new);
+      sum = fmaf(sum, keep, w);
+      acc = fmaf(acc, keep, w * val[q]);
+      M = m_new;
     }
   }
-  __syncthreads();
-  for (int i = tid; i < n * GH; i += blockDim.x) {
-    const int gi = i % GH;
-    wsm[i] = fast_exp2(wsm[i] - mx[gi]) / sm[gi];
-  }
-  __syncthreads();
-  const int gi = tid / D, d = tid - gi * D;
-  const float* po = a.part_o + (slot0 * GH + gi) * D + d;
-  const float* p1 = a.l1_o + ((l1_row + gi) * a.l1_max_chunks) * D + d;
-  const size_t stride = static_cast<size_t>(GH) * D;
-  float o0 = 0.f, o1 = 0.f, o2 = 0.f, o3 = 0.f;
-  int j = 0;
-  auto term = [&](int jj) {  // weight 0 marks a CTA without a partial: skip its stale slot
-    const float w = wsm[jj * GH + gi];
-    if (w == 0.f) return 0.f;
-    return w * (jj < n2 ? po[jj * stride] : p1[static_cast<size_t>(jj - n2) * D]);
-  };
-  for (; j + 4 <= n; j += 4) {
-    o0 += term(j);
-    o1 += term(j + 1);
-    o2 += term(j + 2);
-    o3 += term(j + 3);
-  }
-  for (; j < n; ++j) o0 += term(j);
   const int row = __ldg(a.query_start_loc + s);
   static_cast<T*>(a.out)[(static_cast<size_t>(row) * a.num_q_heads + hg * GH + gi) * D + d] =
-      Elem<T>::narrow((o0 + o1) + (o2 + o3));
+      Elem<T>::narrow(acc / sum);
 }
 
 constexpr int kNCW = 4;
@@ -589,9 +581,8 @@ cudaError_t launch_decode_bs(DecodeArgs& a, const CUtensorMap& kmap, const CUten
 template <typename T, int D, int BS, int GH>
 cudaError_t launch_combine_t(const DecodeArgs& a, cudaStream_t stream) {
   auto kern = decode_combine_kernel<T, D, BS, GH>;
-  const size_t smem = (static_cast<size_t>(a.grid) + a.l1_max_chunks + 2) * GH * sizeof(float);
   const unsigned grid = static_cast<unsigned>(a.num_seqs) * (a.num_q_heads / GH);
-  return launch_chained(kern, dim3(grid), dim3(GH * D), smem, stream, a);
+  return launch_chained(kern, dim3(grid), dim3(GH * D), 0, stream, a);
 }
 
 template <typename T, int D, int BS>
