@@ -69,10 +69,11 @@ def _sources_digest() -> str:
 
 
 def decode_kernel_name(geo) -> str:
-    """The decode kernel libpa picks for this geometry (its policy for a plain
-    pa_attention call: tensor cores for bf16, head_dim 128, groups of 2/4/8)."""
+    """The decode kernel libpa runs for this geometry: the CUDA-core kernel,
+    unless PA_DECODE_TC=1 selects the tensor-core one (bf16, head_dim 128,
+    groups of 2/4/8)."""
     env = os.environ.get("PA_DECODE_TC", "")
-    tc = geo.dtype == "bf16" and geo.head_dim == 128 and geo.group in (2, 4, 8) and env != "0"
+    tc = geo.dtype == "bf16" and geo.head_dim == 128 and geo.group in (2, 4, 8) and env == "1"
     return "paged_decode_tc_kernel" if tc else "paged_decode_kernel"
 
 

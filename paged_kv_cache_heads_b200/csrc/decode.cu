@@ -98,10 +98,15 @@ struct DecodeCfg {
   static size_t smem_bytes(int num_seqs) { return 1024 + kSeqOff + 12ull * (num_seqs + 1); }
 };
 
+#ifndef PA_DECODE_GQA_CTAS_PER_SM
+#define PA_DECODE_GQA_CTAS_PER_SM 3
+#endif
+
 template <typename T, int D, int BS, int GH, int KH, int NCW>
-// Registers are budgeted for 4 (one head) or 3 (grouped heads) CTAs per SM:
-// more resident warps hide the latency of the shuffle and FMA chains.
-__global__ void __launch_bounds__((NCW + 1) * 32, (GH == 1 ? 4 : 3))
+// Registers are budgeted for 4 (one head) or PA_DECODE_GQA_CTAS_PER_SM
+// (grouped heads) CTAs per SM: more resident warps hide the latency of the
+// shuffle and FMA chains.
+__global__ void __launch_bounds__((NCW + 1) * 32, (GH == 1 ? 4 : PA_DECODE_GQA_CTAS_PER_SM))
     paged_decode_kernel(const __grid_constant__ CUtensorMap kmap,
                         const __grid_constant__ CUtensorMap vmap, const DecodeArgs a) {
   using C = DecodeCfg<T, D, BS, GH, KH, NCW>;

@@ -578,12 +578,12 @@ bool decode_tc_supported(int32_t group, const pa_cache_desc& c) {
 }
 
 bool decode_uses_tc(int32_t group, const pa_cache_desc& c, bool short_units) {
-  static const int mode = [] {  // -1: by workload, 0: never, 1: always
+  (void)short_units;
+  static const bool enabled = [] {
     const char* env = getenv("PA_DECODE_TC");
-    return env && (env[0] == '0' || env[0] == '1') ? env[0] - '0' : -1;
+    return env && env[0] == '1';
   }();
-  if (!decode_tc_supported(group, c) || mode == 0) return false;
-  return mode == 1 || !short_units;
+  return enabled && decode_tc_supported(group, c);
 }
 
 cudaError_t launch_decode_tc(DecodeArgs& a, const CUtensorMap& qmap, const CUtensorMap& kmap,

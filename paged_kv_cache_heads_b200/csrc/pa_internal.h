@@ -82,11 +82,13 @@ cudaError_t launch_copy_blocks(const int32_t* pairs, int32_t num_pairs, void* k_
                                cudaStream_t stream);
 cudaError_t launch_decode(DecodeArgs& a, const CUtensorMap& kmap, const CUtensorMap& vmap,
                           const pa_cache_desc& c, cudaStream_t stream);
-// Grouped-query decode on the tensor cores: bf16, head_dim 128, group 2, 4 or 8.
-// It wins on long units (128-token tiles); the CUDA-core kernel streams block
-// by block and wins when units are a few blocks long, as in the suffix pass of
-// cascade decode (`short_units`). Environment PA_DECODE_TC=0 never selects the
-// tensor-core kernel, PA_DECODE_TC=1 always does where supported.
+// Grouped-query decode on the tensor cores: bf16, head_dim 128, group 2, 4 or 8,
+// selected only with environment PA_DECODE_TC=1. Decode runs on the CUDA-core
+// kernel by default: the tensor cores are kept for the dense contractions of
+// prefill and the cascade prefix pass, and with chained launches the CUDA-core
+// grouped kernel matches the tensor-core one on the grouped batches measured
+// (within 5 %, faster on two of three). `short_units` marks the cascade suffix
+// pass (units of a few blocks), where the CUDA-core kernel is also the better fit.
 // `qmap` is q as {head_dim, num_q_heads, num_q_tokens} with box {64, group, 1};
 // the cache maps have box {64, 1, block_size, 1}; all three use the 128-byte swizzle.
 bool decode_tc_supported(int32_t group, const pa_cache_desc& c);

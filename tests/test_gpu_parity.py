@@ -258,9 +258,9 @@ def test_decode_large_logits_trigger_rescale(P):
     _check_attention(got, o.out, W.BF16, "decode rescale")
 
 
-def test_decode_many_sequences_two_stage_ring(P):
-    """4600 short sequences: the per-sequence table in shared memory leaves room
-    for only two 64 KiB stages, which selects the two-stage variant."""
+def test_decode_many_sequences(P):
+    """4600 short sequences: a large per-sequence table in shared memory and
+    thousands of units of one or two blocks."""
     rng = np.random.default_rng(4600)
     n = 4600
     lens = rng.integers(1, 48, size=n)
@@ -270,18 +270,33 @@ def test_decode_many_sequences_two_stage_ring(P):
     _check_attention(got, o.out, W.BF16, "many sequences")
 
 
-_CUDA_CORE_SCRIPT = r'''
+_TENSOR_CORE_SCRIPT = r'''
 import sys, numpy as np, torch
 sys.path.insert(0, sys.argv[1])
 from oracle import scenario as oscen
 from paged_kv_cache_heads_b200 import workloads as W, scenario as gs
 import paged_kv_cache_heads_b200 as P
 worst = 0.0
+cases = []
 for seed, g, bs in [(11, 4, 16), (12, 2, 8), (13, 8, 32)]:
     rng = np.random.default_rng(seed)
     lens = [1, bs + 1, int(rng.integers(600, 1400)), int(rng.integers(2000, 2600))]
     wl = W.random_case(seed, num_seqs=4, q_lens=[1] * 4, ctx_extra=[x - 1 for x in lens], num_kv_heads=2,
                        group=g, head_dim=128, block_size=bs, dtype=W.BF16)
+    cases.append((seed, wl))
+# growing logits (the lazy rescale of l and O^T) and 4600 sequences (whose
+# per-sequence table leaves room for only the two-stage ring)
+wl = W.random_case(4242, num_seqs=5, q_lens=[1] * 5, ctx_extra=[15, 900, 2500, 40, 1300], num_kv_heads=2, group=4,
+                   head_dim=128, block_size=16, dtype=W.BF16)
+for op in wl.ops:
+    if op.k is not None and op.k.size:
+        f = W.bf16_bits_to_f32(op.k)
+        op.k = W.f32_to_bf16_bits(f * np.linspace(0.5, 8.0, f.shape[0], dtype=np.float32)[:, None, None])
+cases.append(("ramp", wl))
+lens = np.random.default_rng(4600).integers(1, 48, size=4600)
+cases.append(("many", W.random_case(4600, num_seqs=4600, q_lens=[1] * 4600, ctx_extra=[int(x) - 1 for x in lens],
+                                    num_kv_heads=1, group=8, head_dim=128, block_size=16, dtype=W.BF16)))
+for seed, wl in cases:
     b = gs.prepare(wl)
     gs.run_step(b)
     torch.cuda.synchronize()
@@ -294,13 +309,13 @@ print("OK", worst)
 '''
 
 
-def test_cuda_core_grouped_decode_still_matches(P):
-    """PA_DECODE_TC=0 keeps the CUDA-core grouped kernel reachable; it must
-    stay within tolerance too (it serves fp32 and head_dim 64)."""
+def test_tensor_core_grouped_decode_matches(P):
+    """PA_DECODE_TC=1 selects the tensor-core grouped decode kernel (the
+    default is the CUDA-core kernel); it must stay within tolerance too."""
     import subprocess
     import sys
     root = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
-    env = dict(os.environ, PA_DECODE_TC="0")
-    r = subprocess.run([sys.executable, "-c", _CUDA_CORE_SCRIPT, root], capture_output=True, text=True, env=env,
+    env = dict(os.environ, PA_DECODE_TC="1")
+    r = subprocess.run([sys.executable, "-c", _TENSOR_CORE_SCRIPT, root], capture_output=True, text=True, env=env,
                        cwd=root, timeout=600)
     assert r.returncode == 0 and "OK" in r.stdout, r.stdout + r.stderr
