@@ -106,6 +106,9 @@ def test_attention_validation():
         _attn(max_query_len=5)                                 # more than num_q_tokens
     _attn(num_seqs=0)                                          # empty batch: no-op
     _attn(num_q_tokens=0)
+    with pytest.raises(P.PAError) as e:
+        _attn(num_seqs=8193, num_q_tokens=8193)                # beyond the 8192-sequence batch limit
+    assert e.value.status == P.PA_ERR_UNSUPPORTED
 
 
 def test_workspace_size_policy():

@@ -270,6 +270,41 @@ def test_decode_many_sequences(P):
     _check_attention(got, o.out, W.BF16, "many sequences")
 
 
+@pytest.mark.parametrize("tc", ["0", "1"])
+def test_decode_at_the_batch_limit(P, tc):
+    """8192 sequences, the largest batch pa_attention takes, on both decode
+    kernels (the tensor-core one in a subprocess, since the choice is read once)."""
+    import subprocess
+    import sys
+    root = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+    code = _LIMIT_SCRIPT
+    env = dict(os.environ, PA_DECODE_TC=tc)
+    r = subprocess.run([sys.executable, "-c", code, root], capture_output=True, text=True, env=env, cwd=root,
+                       timeout=900)
+    assert r.returncode == 0 and "OK" in r.stdout, r.stdout + r.stderr
+
+
+_LIMIT_SCRIPT = r'''
+import sys, numpy as np, torch
+sys.path.insert(0, sys.argv[1])
+from oracle import scenario as oscen
+from paged_kv_cache_heads_b200 import workloads as W, scenario as gs
+import paged_kv_cache_heads_b200 as P
+n = 8192
+lens = np.random.default_rng(8192).integers(1, 40, size=n)
+wl = W.random_case(8192, num_seqs=n, q_lens=[1] * n, ctx_extra=[int(x) - 1 for x in lens], num_kv_heads=2,
+                   group=4, head_dim=128, block_size=16, dtype=W.BF16)
+b = gs.prepare(wl)
+gs.run_step(b)
+torch.cuda.synchronize()
+o = oscen.run(wl, W.sentinel_cache(wl.geometry), W.sentinel_cache(wl.geometry))
+err = np.abs(gs.out_as_f64(b.out, W.BF16) - o.out)
+assert np.isfinite(err).all() and err.max() <= 2e-2 and err.mean() <= 2e-3, (err.max(), err.mean())
+assert P.pa_read_device_flags(clear=True) == 0
+print("OK", float(err.max()))
+'''
+
+
 _TENSOR_CORE_SCRIPT = r'''
 import sys, numpy as np, torch
 sys.path.insert(0, sys.argv[1])
