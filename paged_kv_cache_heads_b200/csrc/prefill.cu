@@ -333,26 +333,27 @@ __global__ void __launch_bounds__(160, 2)
       // With a positive scale the row max is taken on the raw scores and the
       // scale is folded into the exponent's FMA below; the causal mask is
       // applied only on tiles that reach past this row's last visible key.
+      // (four independent max chains instead of one 64-long chain)
       float sc = a.scale_log2;
-      float mx = -CUDART_INF_F;
+      float mq[4] = {-CUDART_INF_F, -CUDART_INF_F, -CUDART_INF_F, -CUDART_INF_F};
       if (sc > 0.f && kbase + kBN - 1 <= lim) {
 #pragma unroll
-        for (int c = 0; c < kBN; ++c) mx = fmaxf(mx, sv[c]);
+        for (int c = 0; c < kBN; ++c) mq[c & 3] = fmaxf(mq[c & 3], sv[c]);
       } else if (sc > 0.f) {
 #pragma unroll
         for (int c = 0; c < kBN; ++c) {
           if (kbase + c > lim) sv[c] = -CUDART_INF_F;
-          mx = fmaxf(mx, sv[c]);
+          mq[c & 3] = fmaxf(mq[c & 3], sv[c]);
         }
       } else {
 #pragma unroll
         for (int c = 0; c < kBN; ++c) {
           sv[c] = (kbase + c <= lim) ? sv[c] * sc : -CUDART_INF_F;
-          mx = fmaxf(mx, sv[c]);
+          mq[c & 3] = fmaxf(mq[c & 3], sv[c]);
         }
         sc = 1.f;  // already scaled
       }
-      mx *= sc;
+      float mx = fmaxf(fmaxf(mq[0], mq[1]), fmaxf(mq[2], mq[3])) * sc;
       // Rescale only when the running max grows by more than 2^8; otherwise
       // keep the old reference so P stays below 2^8 and O needs no update.
       const float m_new = fmaxf(m_used, mx);
@@ -378,6 +379,7 @@ __global__ void __launch_bounds__(160, 2)
       }
       l *= alpha;
       uint8_t* prow = ps + r * 128;
+      float lq[4] = {0.f, 0.f, 0.f, 0.f};  // four independent partial sums of this tile
 #pragma unroll
       for (int c8 = 0; c8 < kBN / 8; ++c8) {
         uint32_t pk[4];
@@ -385,12 +387,13 @@ __global__ void __launch_bounds__(160, 2)
         for (int i = 0; i < 4; ++i) {
           const float p0 = fast_exp2(fmaf(sv[c8 * 8 + 2 * i], sc, -m_used));
           const float p1 = fast_exp2(fmaf(sv[c8 * 8 + 2 * i + 1], sc, -m_used));
-          l += p0 + p1;
+          lq[i] += p0 + p1;
           const __nv_bfloat162 h2 = __floats2bfloat162_rn(p0, p1);
           pk[i] = *reinterpret_cast<const uint32_t*>(&h2);
         }
         *reinterpret_cast<uint4*>(prow + ((c8 ^ (r & 7)) << 4)) = make_uint4(pk[0], pk[1], pk[2], pk[3]);
       }
+      l += (lq[0] + lq[1]) + (lq[2] + lq[3]);
       // zero V rows at or beyond L (stale tail of the last block)
       const int vz0 = it.L - kbase;
       if (vz0 < kBN) {
