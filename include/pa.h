@@ -26,9 +26,15 @@
  *    lengths, copy pairs) live in device memory and cannot be checked before
  *    launch. Kernels range-check each index they use; an out-of-range index
  *    is skipped (no memory access) and a bit is set in the library's device
- *    status word (PA_FLAG_*), read with pa_read_device_flags. No kernel traps.
+ *    status word (PA_FLAG_*), read with pa_get_debug_status (one stream) or
+ *    pa_read_device_flags (whole device). No kernel traps.
  *  - All indices are int32. Block-table rows are padded with -1; a negative
  *    slot means a padding token.
+ *  - Device state: the library looks up the device addresses of its own
+ *    device variables (the status word, the static workspace) once per
+ *    device and keeps them for the life of the process. Do not use the
+ *    library across cudaDeviceReset() or any other teardown of a device's
+ *    primary context: the kept addresses would no longer be mapped.
  */
 #ifndef PA_H_
 #define PA_H_
@@ -208,6 +214,20 @@ pa_status pa_attention_cascade(const void* q, const void* k_cache, const void* v
                                const int32_t* groups, int32_t num_groups, int32_t max_group_size,
                                int32_t max_shared_blocks, float scale, const pa_cache_desc* cache, void* out,
                                void* workspace, size_t workspace_bytes, void* stream);
+
+/*
+ * pa_get_debug_status -- stream-ordered read of the device status word of the
+ * current device: waits for the work queued on `stream` so far (only that
+ * stream), writes the OR of the PA_FLAG_* bits raised since the word was last
+ * cleared to *host_flag (0: no index was out of range and no wait gave up),
+ * then clears the word. Flags raised by kernels on other streams that have not
+ * finished are not waited for; use pa_read_device_flags for a device-wide read.
+ *   stream     cudaStream_t as void* (NULL = legacy default stream)
+ *   host_flag  host out
+ * The index checks it reports are always compiled in (there is no separate
+ * debug build): each index is compared once where it is used.
+ */
+pa_status pa_get_debug_status(void* stream, int32_t* host_flag);
 
 /*
  * pa_read_device_flags -- read (and optionally clear) the device status word

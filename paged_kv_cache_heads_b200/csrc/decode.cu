@@ -12,9 +12,11 @@
 // bandwidth (§"三、连续批处理：让GPU一刻不停" of the first page), which shapes
 // the design.
 //
-// This CUDA-core kernel serves fp32 caches, head_dim 64, ungrouped heads and
-// the suffix pass of cascade decode (short units); grouped bf16 heads of 128
-// run on the tensor cores (decode_tc.cu), with the same partition and merge.
+// This CUDA-core kernel serves every decode call by default: both dtypes,
+// head_dim 64 and 128, grouped and ungrouped heads, and the suffix pass of
+// cascade decode. A tensor-core variant for grouped bf16 heads of 128
+// (decode_tc.cu, same partition and merge) is selected only on request
+// (environment PA_DECODE_TC=1).
 //
 // Design (B200):
 //  * A unit is (sequence, group of GH query heads sharing one KV head); its
@@ -137,6 +139,11 @@ __global__ void __launch_bounds__((NCW + 1) * 32, (GH == 1 ? 4 : PA_DECODE_GQA_C
     tma_prefetch_desc(&kmap);
     tma_prefetch_desc(&vmap);
   }
+  // Chained launch: only the set-up above overlaps the previous grid. Every
+  // input (index arrays, q, the cache) may have been written by the kernel
+  // just before this one on the stream, and its writes are guaranteed
+  // visible only after this wait.
+  grid_dependency_wait();
 
   // ---- decode blocks of every sequence, and their prefix
   int carry = 0;
@@ -166,12 +173,9 @@ __global__ void __launch_bounds__((NCW + 1) * 32, (GH == 1 ? 4 : PA_DECODE_GQA_C
     carry += total;
   }
   __syncthreads();
-  // Chained launch: everything above overlaps the previous grid; the cache
-  // (written by a preceding store) and the workspace (read by a preceding
-  // merge) are touched only after it has completed. Only then may the grids
-  // chained after this one start: they read the same cache, and each of them
-  // waits for its own predecessor at most.
-  grid_dependency_wait();
+  // The grids chained after this one may start now: every input they read
+  // was complete before this grid passed its wait, and each of them waits
+  // for its own predecessor at most.
   launch_dependents();
   const int64_t B = static_cast<int64_t>(prefix[a.num_seqs]) * HG;  // blocks of all units
   if (blockIdx.x == 0 && a.seq_prefix)

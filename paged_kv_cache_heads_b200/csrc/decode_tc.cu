@@ -174,6 +174,11 @@ __global__ void __launch_bounds__(192, 1)
     tma_prefetch_desc(&kmap);
     tma_prefetch_desc(&vmap);
   }
+  // Chained launch: only the set-up above overlaps the previous grid. Every
+  // input (index arrays, q, the cache) may have been written by the kernel
+  // just before this one on the stream, and its writes are guaranteed
+  // visible only after this wait.
+  grid_dependency_wait();
 
   // ---- decode blocks of every sequence, and their prefix
   int carry = 0;
@@ -203,12 +208,9 @@ __global__ void __launch_bounds__(192, 1)
   tc::fence_before_sync();
   __syncthreads();
   tc::fence_after_sync();
-  // Chained launch: everything above overlaps the previous grid; the cache
-  // (written by a preceding store) and the workspace (read by a preceding
-  // merge) are touched only after it has completed. Only then may the grids
-  // chained after this one start: they read the same cache, and each of them
-  // waits for its own predecessor at most.
-  grid_dependency_wait();
+  // The grids chained after this one may start now: every input they read
+  // was complete before this grid passed its wait, and each of them waits
+  // for its own predecessor at most.
   launch_dependents();
   const uint32_t tmem = *tmem_slot;
   const int64_t B = static_cast<int64_t>(prefix[a.num_seqs]) * HG;  // blocks of all units

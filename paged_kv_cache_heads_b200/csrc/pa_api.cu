@@ -610,6 +610,22 @@ pa_status pa_attention_cascade(const void* q, const void* k_cache, const void* v
   return PA_OK;
 }
 
+pa_status pa_get_debug_status(void* stream, int32_t* host_flag) {
+  if (!host_flag) return fail(PA_ERR_INVALID_ARG, "host_flag is NULL");
+  unsigned* word = nullptr;
+  cudaError_t e = status_ptr(&word);
+  if (e != cudaSuccess) return cuda_fail(e, "status word");
+  const cudaStream_t s = static_cast<cudaStream_t>(stream);
+  // Read, then clear, in stream order; only this stream is waited for.
+  unsigned v = 0;
+  e = cudaMemcpyAsync(&v, word, sizeof(v), cudaMemcpyDeviceToHost, s);
+  if (e == cudaSuccess) e = cudaMemsetAsync(word, 0, sizeof(unsigned), s);
+  if (e == cudaSuccess) e = cudaStreamSynchronize(s);
+  if (e != cudaSuccess) return cuda_fail(e, "read status word");
+  *host_flag = static_cast<int32_t>(v);
+  return PA_OK;
+}
+
 pa_status pa_read_device_flags(uint32_t* flags, int32_t clear) {
   if (!flags) return fail(PA_ERR_INVALID_ARG, "flags is NULL");
   cudaError_t e = cudaDeviceSynchronize();

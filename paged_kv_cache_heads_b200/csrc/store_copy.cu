@@ -37,17 +37,22 @@ __global__ void __launch_bounds__(kThreads) store_kv_kernel(
   // A chained attention grid may start its prologue now; it waits for this
   // grid's completion before it reads the cache.
   launch_dependents();
+  // The host guarantees total < 2^32, so every index below total fits in 32
+  // bits; the loop counter itself is 64-bit so that the last step past total
+  // cannot wrap around to a small value.
   const uint32_t per_tensor = num_tokens * n16;
-  const uint32_t total = 2u * per_tensor;
-  const uint32_t stride = gridDim.x * blockDim.x;
-  for (uint32_t base = blockIdx.x * blockDim.x + threadIdx.x; base < total; base += stride * kUnroll) {
+  const uint64_t total = 2ull * per_tensor;
+  const uint64_t stride = static_cast<uint64_t>(gridDim.x) * blockDim.x;
+  for (uint64_t base = static_cast<uint64_t>(blockIdx.x) * blockDim.x + threadIdx.x; base < total;
+       base += stride * kUnroll) {
     uint4 r[kUnroll];
     uint4* dst[kUnroll];
 #pragma unroll
     for (int u = 0; u < kUnroll; ++u) {
       dst[u] = nullptr;
-      const uint32_t i = base + u * stride;
-      if (i < total) {
+      const uint64_t i64 = base + u * stride;
+      if (i64 < total) {
+        const uint32_t i = static_cast<uint32_t>(i64);
         const bool is_v = i >= per_tensor;
         const uint32_t j = is_v ? i - per_tensor : i;
         const uint32_t t = j / n16;

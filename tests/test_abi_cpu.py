@@ -78,6 +78,30 @@ def test_store_and_copy_validation():
         P.pa_copy_blocks(None, 3, FAKE, FAKE, DESC, stream=0)
 
 
+def test_store_size_guard_boundary():
+    """The store kernel indexes its 16-byte vectors with 32-bit integers, so
+    pa_store_kv refuses calls of 2^32 vectors or more before launching
+    anything: 8 KV heads x 128 bf16 columns are 128 vectors per row and
+    token, 256 per token for K and V, so 2^24 tokens are exactly 2^32 vectors."""
+    n16 = 8 * 128 * 2 // 16
+    limit = (1 << 32) // (2 * n16)
+    assert 2 * limit * n16 == 1 << 32
+    with pytest.raises(P.PAError) as e:
+        P.pa_store_kv(FAKE, FAKE, FAKE, limit, FAKE, FAKE, DESC, stream=0)
+    assert e.value.status == P.PA_ERR_UNSUPPORTED and "too large" in str(e.value)
+    with pytest.raises(P.PAError) as e:
+        P.pa_store_kv(FAKE, FAKE, FAKE, limit + 1, FAKE, FAKE, DESC, stream=0)
+    assert e.value.status == P.PA_ERR_UNSUPPORTED
+    import torch
+    if torch.cuda.is_available():
+        return  # one token fewer passes the guard and would launch on these fake pointers
+    # one token fewer passes the size guard; without a GPU the call then fails
+    # at the first CUDA call, not at the guard
+    with pytest.raises(P.PAError) as e:
+        P.pa_store_kv(FAKE, FAKE, FAKE, limit - 1, FAKE, FAKE, DESC, stream=0)
+    assert e.value.status == P.PA_ERR_CUDA
+
+
 def _attn(**kw):
     args = dict(q=FAKE, k_cache=FAKE, v_cache=FAKE, block_tables=FAKE, max_blocks_per_seq=128,
                 context_lens=FAKE, query_start_loc=FAKE, num_seqs=4, num_q_tokens=4, num_q_heads=32,

@@ -296,6 +296,31 @@ def test_stats_paged_vs_preallocated_fragmentation_on_decode_batch():
     assert pre == pytest.approx(1 - st["tokens"] / (len(wl.batch_seqs) * 2048), abs=1e-15)
 
 
+def test_preallocation_fragmentation_pinned_to_the_pages_example(golden):
+    """[C] §"二、KV Cache管理：从浪费到极致复用": a request that generates 50 tokens
+    under a scheme that reserves 2048 slots per request leaves 1998 of its
+    2048 slots unused (worked by hand: 2048 - 50 = 1998)."""
+    ex = golden["short_generation"]
+    n, reserved = ex["generated_tokens"], ex["preallocated_tokens"]
+    assert (n, reserved) == (50, 2048)
+    assert oracle.preallocation_fragmentation([n], reserved) == 1998 / 2048
+    # a second request that fills its whole reservation wastes nothing:
+    # 1998 unused slots out of 2 x 2048 reserved
+    assert oracle.preallocation_fragmentation([n, reserved], reserved) == 1998 / 4096
+    # closed forms: every request full -> 0; no tokens at all -> 1
+    assert oracle.preallocation_fragmentation([reserved] * 3, reserved) == 0.0
+    assert oracle.preallocation_fragmentation([0, 0], reserved) == 1.0
+
+
+def test_preallocation_fragmentation_planted_slip_fails():
+    """Dividing by the batch's longest request instead of the reservation (a
+    plausible slip) gives 1/4 here, not 1 - 150/4096."""
+    lens = [50, 100]
+    slip = 1.0 - sum(lens) / (len(lens) * max(lens))
+    assert slip == 0.25
+    assert oracle.preallocation_fragmentation(lens, 2048) == 1.0 - 150 / 4096 != slip
+
+
 def test_stats_count_planted_double_counting():
     """A plausible slip, counting a shared slot once per holder, breaks the fork pin."""
     bm = BlockManager(8, 4)
