@@ -213,11 +213,12 @@ def step_work(wl, step_tokens: int, step_pairs: int):
 
 
 def launches_per_step(b) -> int:
-    """Kernels one step launches: store, copy (if pairs), decode + split merge, prefill (if q_len > 1)."""
+    """Kernels one step launches: store, copy (if pairs), decode + split merge,
+    prefill + its merge (if q_len > 1)."""
     wl = b.wl
     n = (1 if b.num_step_tokens else 0) + (1 if b.step_pairs.shape[0] else 0) + 2
     if wl.max_query_len > 1:
-        n += 1
+        n += 2
     return n
 
 
@@ -329,19 +330,30 @@ def measure_ours(wl, steps: int, warmup: int, device, gpu_index: int):
     attn_ms = [a.elapsed_time(z) for a, z in ev]
 
     # ---- the same device-resident step replayed from a CUDA graph (no host launch gaps)
+    # K steps are timed, bracketed by a barrier and a synchronize; the K-step
+    # measurement is repeated for about a second so the clock samples cover a
+    # long stretch under load, and the median repeat is reported.
     graph = gs.capture_step(b)
     for _ in range(max(warmup, 1)):
         graph.replay()
     torch.cuda.synchronize(device)
-    barrier()
-    with ClockSampler(gpu_index) as clocks_g:
+
+    def graph_steps():
+        barrier()
+        torch.cuda.synchronize(device)
         start.record(stream)
         for _ in range(steps):
             graph.replay()
         end.record(stream)
         torch.cuda.synchronize(device)
-    barrier()
-    ms_graph = start.elapsed_time(end)
+        barrier()
+        return start.elapsed_time(end)
+
+    with ClockSampler(gpu_index) as clocks_g:
+        first = graph_steps()
+        repeats = int(min(500, max(1, reduce_max(float(np.ceil(1000.0 / max(first, 1e-3))), device))))
+        graph_reps = [first] + [graph_steps() for _ in range(repeats - 1)]
+    ms_graph = statistics.median(graph_reps)
     del graph
     ms_total = min(ms_eager, ms_graph)
     if ms_graph <= ms_eager:
@@ -395,7 +407,7 @@ def measure_ours(wl, steps: int, warmup: int, device, gpu_index: int):
     flags = P.pa_read_device_flags(clear=True)
     return dict(bm_stats=bm_stats, kernels=kernels, step_mode="cuda_graph" if ms_graph <= ms_eager else "eager",
                 step_eager_ms=ms_eager / steps, step_graph_ms=ms_graph / steps, e2e_eager_ms=e2e_eager_ms, e2e_graph_ms=e2e_graph_ms, ms_total=ms_total, attn_ms=attn_ms, e2e_ms=e2e_ms, h2d=h2d, d2h=d2h, clocks=clocks.summary(),
-                launches=launches_per_step(b) * steps, step_tokens=b.num_step_tokens,
+                launches=launches_per_step(b) * steps, timed_repeats=len(graph_reps), step_tokens=b.num_step_tokens,
                 step_pairs=int(b.step_pairs.shape[0]), flags=flags, max_context_len=b.max_context_len)
 
 
@@ -457,26 +469,11 @@ def measure_kernels(b, reps: int = 10):
         ms = timed(lambda: P.pa_copy_blocks(pairs, npairs, b.k_cache, b.v_cache, b.desc), "pa_copy")
         by = 4 * npairs * geo.block_size * row
         res["copy"] = {"pairs": npairs, "launch_ms": ms, "algorithmic_bytes": by, "gbs": by / (ms * 1e-3) / 1e9}
-    pre = [i for i, q in enumerate(wl.q_lens) if q > 1]
-    if pre and pre == list(range(len(pre))):
-        qsl = b.host["query_start_loc"][: len(pre) + 1]
-        t = int(qsl[-1])
-        lens = b.host["context_lens"][: len(pre)]
-        ctx = int(lens.max())
-        mq = int(max(wl.q_lens[i] for i in pre))
-        ws_b = P.pa_attention_workspace_size(len(pre), geo.num_q_heads, mq, ctx, b.desc)
-        ws = torch.empty(max(ws_b, 16), dtype=torch.uint8, device=dev)
-        bt, cl, qs = b.block_tables[: len(pre)].contiguous(), b.context_lens[: len(pre)].contiguous(), \
-            torch.from_numpy(qsl).to(dev)
-        out = torch.empty_like(b.out)
-        ms = timed(lambda: P.pa_attention(b.q, b.k_cache, b.v_cache, bt, geo.max_blocks_per_seq, cl, qs, len(pre),
-                                          t, geo.num_q_heads, mq, ctx, wl.scale, b.desc, out, ws, ws_b),
-                   "pa_prefill_only")
-        flops = 0
-        for i in pre:
-            L, ql = int(lens[i]), wl.q_lens[i]
-            flops += 4 * geo.head_dim * geo.num_q_heads * sum(L - ql + j + 1 for j in range(ql))
-        res["prefill_only"] = {"seqs": len(pre), "q_tokens": t, "launch_ms": ms, "flops": flops,
+    po = prefill_only_call(b)
+    if po is not None:
+        fn, flops, npre, t = po
+        ms = timed(fn, "pa_prefill_only")
+        res["prefill_only"] = {"seqs": npre, "q_tokens": t, "launch_ms": ms, "flops": flops,
                                "tflops": flops / (ms * 1e-3) / 1e12}
     # cascade: when sequences of the batch share leading blocks, the same
     # attention with each group's shared blocks read once
@@ -512,6 +509,118 @@ def measure_kernels(b, reps: int = 10):
     return res
 
 
+def prefill_only_call(b):
+    """pa_attention over the batch's leading sequences with q_len > 1 alone:
+    (call, algorithmic flops, sequences, query tokens), or None."""
+    import torch
+    import paged_kv_cache_heads_b200 as P
+    wl, geo = b.wl, b.wl.geometry
+    pre = [i for i, q in enumerate(wl.q_lens) if q > 1]
+    if not pre or pre != list(range(len(pre))):
+        return None
+    dev = b.k_cache.device
+    qsl = b.host["query_start_loc"][: len(pre) + 1]
+    t = int(qsl[-1])
+    lens = b.host["context_lens"][: len(pre)]
+    ctx = int(lens.max())
+    mq = int(max(wl.q_lens[i] for i in pre))
+    ws_b = P.pa_attention_workspace_size(len(pre), geo.num_q_heads, mq, ctx, b.desc)
+    ws = torch.empty(max(ws_b, 16), dtype=torch.uint8, device=dev)
+    bt, cl, qs = b.block_tables[: len(pre)].contiguous(), b.context_lens[: len(pre)].contiguous(), \
+        torch.from_numpy(qsl).to(dev)
+    out = torch.empty_like(b.out)
+    flops = 0
+    for i in pre:
+        L, ql = int(lens[i]), wl.q_lens[i]
+        flops += 4 * geo.head_dim * geo.num_q_heads * sum(L - ql + j + 1 for j in range(ql))
+
+    def fn():
+        P.pa_attention(b.q, b.k_cache, b.v_cache, bt, geo.max_blocks_per_seq, cl, qs, len(pre), t,
+                       geo.num_q_heads, mq, ctx, wl.scale, b.desc, out, ws, ws_b)
+    return fn, flops, len(pre), t
+
+
+# --------------------------------------------------------------------------
+# every configuration: one attention call at a time, L2 flushed before each
+# --------------------------------------------------------------------------
+
+SWEEP = ("tiny", "gqa_long", "prefix_cow", "mixed_bs8", "mixed_bs16", "mixed_bs32")
+L2_FLUSH_BYTES = 512 << 20   # > 4x the 126 MB L2
+
+
+def timed_calls(fn, reps: int, flush=None):
+    """Each of ``reps`` calls timed alone with CUDA events on the current
+    stream; before each one ``flush`` (a write of L2_FLUSH_BYTES) evicts the L2,
+    outside the timed interval. Returns median / p10 / p90 in ms."""
+    import torch
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(reps)]
+    fn()
+    torch.cuda.synchronize()
+    for i in range(reps):
+        if flush is not None:
+            flush.fill_(i & 0x7F)
+        ev[i][0].record()
+        fn()
+        ev[i][1].record()
+    torch.cuda.synchronize()
+    t = sorted(a.elapsed_time(z) for a, z in ev)
+    return {"median_ms": t[len(t) // 2], "p10_ms": t[len(t) // 10], "p90_ms": t[(9 * len(t)) // 10], "reps": reps}
+
+
+def measure_config(name: str, hbm_peak: float, bf16_peak: float, flush, reps: int = 30, oracle: bool = True):
+    """Attention call of one configuration (L2 cold), its prefill rows alone,
+    its cascade call when sequences share a prompt, and one oracle step."""
+    import torch
+    import paged_kv_cache_heads_b200 as P
+    from paged_kv_cache_heads_b200 import scenario as gs
+    wl = build_workload(name)
+    geo = wl.geometry
+    b = gs.prepare(wl)
+    gs.run_step(b)
+    torch.cuda.synchronize()
+    work = step_work(wl, b.num_step_tokens, int(b.step_pairs.shape[0]))
+    t = timed_calls(lambda: gs.run_attention(b), reps, flush)
+    ms = t["median_ms"]
+    ent = {"attention_us": ms * 1e3, "p10_us": t["p10_ms"] * 1e3, "p90_us": t["p90_ms"] * 1e3, "reps": reps,
+           "query_tokens_per_s": wl.num_q_tokens / (ms * 1e-3), "algorithmic_bytes": work["attn_bytes"],
+           "gbs": work["attn_bytes"] / (ms * 1e-3) / 1e9,
+           "frac_of_hbm_peak": work["attn_bytes"] / (ms * 1e-3) / 1e9 / hbm_peak,
+           "l2": "flushed before each call (%d MB write)" % (L2_FLUSH_BYTES >> 20)}
+    e = 2 if geo.dtype == "bf16" else 4
+    tok_bytes = 2 * geo.num_kv_heads * geo.head_dim * e
+    lens = b.host["context_lens"]
+    po = prefill_only_call(b)
+    if po is not None:
+        fn, flops, npre, qt = po
+        tp = timed_calls(fn, reps, flush)
+        ent["prefill_only"] = {"seqs": npre, "q_tokens": qt, "flops": flops, "us": tp["median_ms"] * 1e3,
+                               "tflops": flops / (tp["median_ms"] * 1e-3) / 1e12,
+                               "frac_of_bf16_peak": flops / (tp["median_ms"] * 1e-3) / 1e12 / bf16_peak}
+    plan = gs.plan_cascade(b) if all(q == 1 for q in wl.q_lens) else None
+    if plan is not None and plan.num_groups:
+        out = torch.empty_like(b.out)
+        tc_ = timed_calls(lambda: gs.run_attention_cascade(b, plan, out=out), reps, flush)
+        shared, groups = plan.host["shared"], plan.host["groups"]
+        own = sum(int(L) - int(sh) * geo.block_size for L, sh in zip(lens, shared))
+        once = sum(int(shared[f]) * geo.block_size for f, _ in groups)
+        unique = (own + once) * tok_bytes
+        cms = tc_["median_ms"]
+        ent["cascade"] = {"us": cms * 1e3, "kv_bytes_read": unique, "kv_bytes_logical": int(np.sum(lens)) * tok_bytes,
+                          "gbs": unique / (cms * 1e-3) / 1e9, "frac_of_hbm_peak": unique / (cms * 1e-3) / 1e9 / hbm_peak}
+        # the plain call reads every distinct block from HBM once as well
+        # (shared ones are L2 hits after the first read)
+        ent["unique_kv_bytes"] = unique
+        ent["frac_of_hbm_peak_unique"] = (unique + work["attn_bytes"] - work["attn_kv_bytes"]) / (ms * 1e-3) / 1e9 \
+            / hbm_peak
+    ent["device_flags"] = P.pa_read_device_flags(clear=True)
+    del b
+    torch.cuda.empty_cache()
+    if oracle:
+        cpu, _ = time_oracle(wl, budget_s=0.0, min_steps=1, max_steps=1)
+        ent["oracle"] = {"query_tokens_per_s": cpu["value"], "cores": cpu["cores"], "sample": cpu["sample"]}
+    return ent
+
+
 def workload_config(wl, world: int, l2_note: str):
     geo = wl.geometry
     lens = wl.notes["context_lens"]
@@ -537,6 +646,8 @@ def main():
     ap.add_argument("--workload", default="llama7b")
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-sweep", action="store_true",
+                    help="skip the per-configuration sweep that the default workload adds at N=1")
     args = ap.parse_args()
     world, rank, local = dist_env()
     hbm_peak, bf16_peak, peak_src = measured_peaks()
@@ -588,6 +699,19 @@ def main():
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         cpu, _ = time_oracle(wl, budget_s=12.0)
 
+    # every other configuration, one attention call at a time (N=1 only)
+    configs = None
+    if world == 1 and args.workload == "llama7b" and not args.no_sweep:
+        import torch
+        flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=device)
+        configs = {}
+        with ClockSampler(gpu_index) as sweep_clocks:
+            for name in SWEEP:
+                configs[name] = measure_config(name, hbm_peak, bf16_peak, flush,
+                                               oracle=not args.no_cpu_baseline)
+        configs["clocks"] = sweep_clocks.summary()
+        del flush
+
     if world > 1:
         import torch.distributed as dist
         dist.destroy_process_group()
@@ -596,7 +720,11 @@ def main():
     roof = {"kernel": "pa_attention (%s + decode_combine_kernel%s)"
                       % (decode_kernel_name(wl.geometry), " + paged_prefill_kernel" if wl.max_query_len > 1 else ""),
             "bound": "hbm", "achieved": achieved, "peak": hbm_peak, "unit": "GB/s",
-            "frac": achieved / hbm_peak, "traffic": traffic, "peak_source": peak_src + " (MEASURED_PEAKS.json hbm_gbs)"
+            "frac": achieved / hbm_peak, "traffic": traffic,
+            "traffic_source": ("dram__bytes_read.sum + dram__bytes_write.sum of the decode kernel from one ncu "
+                               "capture of this workload (profiles/), decode sources digest %s" % digest)
+            if traffic is not None else "none: the decode kernel sources differ from the captured ones",
+            "peak_source": peak_src + " (MEASURED_PEAKS.json hbm_gbs)"
             if peak_src == "measured" else "fallback 6.65 TB/s",
             "algorithmic_bytes_per_launch": work["attn_bytes"], "launch_ms": attn_ms,
             "kv_read_gbs": work["attn_kv_bytes"] / (attn_ms * 1e-3) / 1e9}
@@ -621,10 +749,13 @@ def main():
                     "graph_ms_per_step": r["e2e_graph_ms"] / args.steps},
             "step_launch": {"mode": r["step_mode"], "eager_ms_per_step": r["step_eager_ms"],
                             "graph_ms_per_step": r["step_graph_ms"]},
-            "gpu_launches": r["launches"], "clocks": r["clocks"], "device_flags": r["flags"],
+            "gpu_launches": r["launches"] * r["timed_repeats"], "timed_repeats": r["timed_repeats"],
+            "clocks": r["clocks"], "device_flags": r["flags"],
             "kernels": kern,
             "block_manager": {k: (round(v, 6) if isinstance(v, float) else v) for k, v in r["bm_stats"].items()},
             "step_bytes": work["attn_bytes"] + work["store_bytes"] + work["copy_bytes"]}
+    if configs is not None:
+        line["configs"] = configs
     print(json.dumps(line), flush=True)
     return 0
 

@@ -237,6 +237,19 @@ pa_status pa_get_debug_status(void* stream, int32_t* host_flag);
  */
 pa_status pa_read_device_flags(uint32_t* flags, int32_t clear);
 
+/*
+ * pa_set_wait_limit_ns -- bound, in nanoseconds, of every device-side wait of
+ * the kernels launched from now on (a consumer waiting for a copy, a producer
+ * waiting for a free stage, a softmax warp waiting for an MMA). A wait that
+ * runs out raises PA_FLAG_WAIT_TIMEOUT and its kernel winds down: its results
+ * are unspecified, but every copy and MMA the kernel issued is waited for
+ * (with the default bound) before its CTA exits, and the device stays usable.
+ * Default 2 s (2000000000); 0 gives up on any wait not already satisfied,
+ * which only a test of the timeout path wants. Process-wide, all devices.
+ * Returns the previous limit.
+ */
+uint64_t pa_set_wait_limit_ns(uint64_t limit_ns);
+
 /* Message for the calling thread's last non-OK status ("" if none). */
 const char* pa_last_error(void);
 

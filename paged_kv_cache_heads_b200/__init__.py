@@ -20,7 +20,7 @@ __all__ = [
     "PAError", "PA_FP32", "PA_BF16", "PA_FLAG_SLOT_RANGE", "PA_FLAG_BLOCK_RANGE",
     "PA_FLAG_CONTEXT_RANGE", "PA_FLAG_PAIR_RANGE", "PA_FLAG_WAIT_TIMEOUT", "CacheDesc",
     "library_path", "load_library", "exported_symbols", "pa_store_kv", "pa_copy_blocks",
-    "pa_attention", "pa_attention_workspace_size", "pa_attention_static_workspace", "pa_read_device_flags", "pa_get_debug_status", "pa_last_error",
+    "pa_attention", "pa_attention_workspace_size", "pa_attention_static_workspace", "pa_read_device_flags", "pa_get_debug_status", "pa_set_wait_limit_ns", "pa_last_error",
     "pa_version", "BlockManager",
 ]
 
@@ -70,6 +70,7 @@ _SIGNATURES = {
                                                  C.c_float, C.POINTER(CacheDesc), _P, _P]),
     "pa_read_device_flags": (C.c_int, [C.POINTER(C.c_uint32), _I32]),
     "pa_get_debug_status": (C.c_int, [_P, C.POINTER(C.c_int32)]),
+    "pa_set_wait_limit_ns": (C.c_uint64, [C.c_uint64]),
     "pa_last_error": (C.c_char_p, []),
     "pa_version": (C.c_char_p, []),
     "pa_bm_create": (C.c_int, [_I32, _I32, _PI32, C.POINTER(_P)]),
@@ -254,6 +255,11 @@ def pa_read_device_flags(clear: bool = True) -> int:
     v = C.c_uint32(0)
     _check(load_library().pa_read_device_flags(C.byref(v), 1 if clear else 0))
     return int(v.value)
+
+
+def pa_set_wait_limit_ns(limit_ns: int) -> int:
+    """Bound of the kernels' device-side waits from now on; returns the previous one."""
+    return int(load_library().pa_set_wait_limit_ns(int(limit_ns)))
 
 
 def pa_get_debug_status(stream=None) -> int:

@@ -231,7 +231,7 @@ __global__ void __launch_bounds__((NCW + 1) * 32, (GH == 1 ? 4 : PA_DECODE_GQA_C
           int good = 1;
           if (lane == 0) {
             const uint32_t st = k % C::kNST, use = k / C::kNST;
-            good = mbar_wait(&empty[st], (use & 1) ^ 1, a.status);
+            good = mbar_wait(&empty[st], (use & 1) ^ 1, a.status, a.wait_limit_ns);
             if (good) {
               uint8_t* dst = smem + st * C::kStageB;
               mbar_arrive_expect_tx(&full[st], C::kStageB);
@@ -247,6 +247,12 @@ __global__ void __launch_bounds__((NCW + 1) * 32, (GH == 1 ? 4 : PA_DECODE_GQA_C
       ids = nids;
       b = bn;
     }
+    // Every load this warp issued lands before it exits (the last one of each
+    // stage; default bound), so no copy is still writing into shared memory
+    // when the CTA exits, even if the consumers gave up early.
+    if (lane == 0)
+      for (uint32_t i = k > static_cast<uint32_t>(C::kNST) ? k - C::kNST : 0; i < k; ++i)
+        mbar_drain(&full[i % C::kNST], (i / C::kNST) & 1, a.status);
     return;
   }
 
@@ -290,7 +296,7 @@ __global__ void __launch_bounds__((NCW + 1) * 32, (GH == 1 ? 4 : PA_DECODE_GQA_C
     for (int i = first; i < nblk; i += (KH > 1 ? 1 : NCW)) {
       const uint32_t kk = k + i;
       const uint32_t st = kk % C::kNST;
-      if (!mbar_wait(&full[st], (kk / C::kNST) & 1, a.status)) { ok = false; break; }
+      if (!mbar_wait(&full[st], (kk / C::kNST) & 1, a.status, a.wait_limit_ns)) { ok = false; break; }
       const uint8_t* Ks = smem + st * C::kStageB + (KH > 1 ? warp * C::kRowB : 0);
       const uint8_t* Vs = Ks + BS * C::kTokB;
       const int tok0 = (g.skip + blo + i) * BS;

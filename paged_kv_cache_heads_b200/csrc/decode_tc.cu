@@ -233,7 +233,7 @@ __global__ void __launch_bounds__(192, 1)
         last_seg = it.seg;
         const uint32_t j = static_cast<uint32_t>(it.seg);
         if (lane == 0) {
-          ok = mbar_wait(&q_empty[j & 1], ((j >> 1) & 1) ^ 1, a.status);
+          ok = mbar_wait(&q_empty[j & 1], ((j >> 1) & 1) ^ 1, a.status, a.wait_limit_ns);
           if (ok) {
             uint8_t* qs = smem + C::kQOff + (j & 1) * C::kQB;
             const int row = __ldg(a.query_start_loc + g.s);
@@ -257,7 +257,7 @@ __global__ void __launch_bounds__(192, 1)
       }
       const uint32_t st = i % NST;
       if (lane == 0) {
-        ok = mbar_wait(&empty[st], ((i / NST) & 1) ^ 1, a.status);
+        ok = mbar_wait(&empty[st], ((i / NST) & 1) ^ 1, a.status, a.wait_limit_ns);
         if (ok) mbar_arrive_expect_tx(&full[st], C::kStageB);
       }
       ok = __shfl_sync(0xffffffffu, ok, 0) != 0;
@@ -275,9 +275,9 @@ __global__ void __launch_bounds__(192, 1)
     // wait (bounded) for the last use of every stage and Q buffer.
     if (lane == 0) {
       for (uint32_t k = i > NST ? i - NST : 0; k < i; ++k)
-        if (!mbar_wait(&full[k % NST], (k / NST) & 1, a.status)) break;
+        if (!mbar_drain(&full[k % NST], (k / NST) & 1, a.status)) break;
       for (int j = last_seg - 1; j <= last_seg; ++j)
-        if (j >= 0 && !mbar_wait(&q_full[j & 1], (j >> 1) & 1, a.status)) break;
+        if (j >= 0 && !mbar_drain(&q_full[j & 1], (j >> 1) & 1, a.status)) break;
     }
     __syncwarp();
   } else if (warp == 5) {
@@ -342,7 +342,7 @@ __global__ void __launch_bounds__(192, 1)
           const uint64_t now = globaltimer_ns();
           if (t0 == 0) {
             t0 = now;
-          } else if (now - t0 > PA_WAIT_LIMIT_NS || flag_raised(a.status, PA_FLAG_WAIT_TIMEOUT)) {
+          } else if (now - t0 >= a.wait_limit_ns || flag_raised(a.status, PA_FLAG_WAIT_TIMEOUT)) {
             raise_flag(a.status, PA_FLAG_WAIT_TIMEOUT);
             ok = false;
           }
@@ -350,7 +350,7 @@ __global__ void __launch_bounds__(192, 1)
       }
       // no MMA may be in flight when TMEM is released
       tc::commit(mma_done);
-      mbar_wait(mma_done, 0, a.status);
+      mbar_drain(mma_done, 0, a.status);
     }
     __syncwarp();
   } else {
@@ -374,7 +374,7 @@ __global__ void __launch_bounds__(192, 1)
       }
       const int tok = (g.skip + it.tb) * BS + tid;
       const bool valid = tok < lim;
-      failed = failed || !mbar_wait(&s_full[b], (i >> 1) & 1, a.status);
+      failed = failed || !mbar_wait(&s_full[b], (i >> 1) & 1, a.status, a.wait_limit_ns);
       failed = __any_sync(0xffffffffu, failed);
       float sv[GH];
       if (!failed) {
@@ -415,7 +415,7 @@ __global__ void __launch_bounds__(192, 1)
         if (any_fail) break;  // the same decision in every softmax thread
         if (!it.first()) {
           // O^T holds the P.V products up to tile i-1: wait for them, then rescale
-          failed = !mbar_wait(&pv_done[(i - 1) & 1], ((i - 1) >> 1) & 1, a.status);
+          failed = !mbar_wait(&pv_done[(i - 1) & 1], ((i - 1) >> 1) & 1, a.status, a.wait_limit_ns);
           failed = __any_sync(0xffffffffu, failed);
           if (!failed) {
             tc::fence_after_sync();
@@ -437,7 +437,7 @@ __global__ void __launch_bounds__(192, 1)
       }
       // P^T buffer b was last read by the P.V MMA of tile i-2
       if (i >= 2) {
-        failed = failed || !mbar_wait(&pv_done[b], ((i - 2) >> 1) & 1, a.status);
+        failed = failed || !mbar_wait(&pv_done[b], ((i - 2) >> 1) & 1, a.status, a.wait_limit_ns);
         failed = __any_sync(0xffffffffu, failed);
       }
       if (!failed) {
@@ -449,7 +449,7 @@ __global__ void __launch_bounds__(192, 1)
         // a V row past L inside a loaded block holds stale bits: zero it
         if (tok >= L && tid < it.blocks() * BS) {
           const uint32_t st = i % NST;
-          if (mbar_wait(&full[st], (i / NST) & 1, a.status)) {
+          if (mbar_wait(&full[st], (i / NST) & 1, a.status, a.wait_limit_ns)) {
             uint8_t* vrow = smem + st * C::kStageB + C::kKB + tid * 128;
 #pragma unroll
             for (int c = 0; c < 8; ++c) {
@@ -466,7 +466,7 @@ __global__ void __launch_bounds__(192, 1)
 
       if (it.last()) {
         // ---- segment epilogue: O^T / l to the output rows or this CTA's partial
-        failed = failed || !mbar_wait(&pv_done[b], (i >> 1) & 1, a.status);
+        failed = failed || !mbar_wait(&pv_done[b], (i >> 1) & 1, a.status, a.wait_limit_ns);
         failed = __any_sync(0xffffffffu, failed);
         float ov[GH];
         if (!failed) {

@@ -2,6 +2,7 @@
 // status word, and dispatch to the kernels. See include/pa.h for the contract
 // of every entry point.
 #include <algorithm>
+#include <atomic>
 #include <cuda.h>
 #include <cuda_runtime.h>
 
@@ -177,6 +178,12 @@ constexpr int32_t kMaxSeqs = 8192;
 
 void set_last_error(const char* msg) { g_last_error = msg; }
 
+namespace {
+std::atomic<uint64_t> g_wait_limit_ns{PA_WAIT_LIMIT_NS};
+}  // namespace
+
+uint64_t wait_limit_ns() { return g_wait_limit_ns.load(std::memory_order_relaxed); }
+
 int32_t ctas_per_sm(const void* kernel, int threads, size_t smem, int cap) {
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess) return 1;
@@ -309,6 +316,9 @@ pa_status launch_decode_path(DecodeArgs& a, const void* q, const void* k_cache, 
 // per-sequence decode block prefix. False for arguments the size query cannot use.
 struct WorkspaceLayout {
   size_t bytes = 0, lse_off = 0, prefix_off = 0;
+  // prefill rows: partition, partial outputs and their log-sum-exp
+  size_t pf_prefix_off = 0, pf_o_off = 0, pf_lse_off = 0;
+  int32_t pf_grid = 0;
 };
 bool workspace_layout(int32_t num_seqs, int32_t num_q_heads, int32_t max_query_len, int32_t max_context_len,
                       const pa_cache_desc* cache, WorkspaceLayout* w) {
@@ -329,6 +339,15 @@ bool workspace_layout(int32_t num_seqs, int32_t num_q_heads, int32_t max_query_l
   w->lse_off = (parts * cache->head_dim * 4 + 255) & ~size_t(255);
   w->prefix_off = (w->lse_off + parts * 4 + 255) & ~size_t(255);
   w->bytes = w->prefix_off + (size_t(num_seqs) + 1) * 4;
+  if (max_query_len > 1 && cache->dtype == PA_BF16) {
+    // two partial slots of 256 rows per prefill CTA
+    w->pf_grid = prefill_grid(num_seqs, num_q_heads, cache->num_kv_heads, max_query_len, max_context_len);
+    const size_t rows = size_t(2) * w->pf_grid * 256;
+    w->pf_prefix_off = (w->bytes + 255) & ~size_t(255);
+    w->pf_o_off = (w->pf_prefix_off + (size_t(num_seqs) + 3) * 4 + 255) & ~size_t(255);
+    w->pf_lse_off = (w->pf_o_off + rows * cache->head_dim * 4 + 255) & ~size_t(255);
+    w->bytes = w->pf_lse_off + rows * 4;
+  }
   return true;
 }
 }  // namespace
@@ -367,6 +386,12 @@ pa_status pa_attention(const void* q, const void* k_cache, const void* v_cache,
     return fail(PA_ERR_UNSUPPORTED, "max_blocks_per_seq too large");
   if (max_query_len > 1 && cache->dtype != PA_BF16)
     return fail(PA_ERR_UNSUPPORTED, "query rows with q_len > 1 need a bf16 cache");
+  if (max_query_len > 1) {
+    // the prefill grid numbers key tiles of (token pair, head group) items in int32
+    const int64_t gh = prefill_heads_per_tile(num_q_heads / cache->num_kv_heads);
+    const int64_t tiles = (int64_t(num_q_tokens) / 2 + 1) * (num_q_heads / gh) * ((int64_t(max_context_len) + 63) / 64);
+    if (tiles >= (1ll << 31)) return fail(PA_ERR_UNSUPPORTED, "prefill batch too large; split it");
+  }
   if (!(scale == scale)) return fail(PA_ERR_INVALID_ARG, "scale is NaN");
 
   WorkspaceLayout wl;
@@ -403,6 +428,7 @@ pa_status pa_attention(const void* q, const void* k_cache, const void* v_cache,
   a.grid = 0;
   a.hpu = 1;
   a.scale_log2 = scale_log2;
+  a.wait_limit_ns = wait_limit_ns();
   a.skip_blocks = nullptr;
   a.l1_o = nullptr;
   a.l1_lse = nullptr;
@@ -433,6 +459,7 @@ pa_status pa_attention(const void* q, const void* k_cache, const void* v_cache,
     p.max_query_len = max_query_len;
     p.num_q_tokens = num_q_tokens;
     p.scale_log2 = scale_log2;
+    p.wait_limit_ns = wait_limit_ns();
     p.groups = nullptr;
     p.skip_blocks = nullptr;
     p.num_groups = 0;
@@ -440,6 +467,10 @@ pa_status pa_attention(const void* q, const void* k_cache, const void* v_cache,
     p.l1_lse = nullptr;
     p.l1_max_chunks = 0;
     p.l1_chunk_blocks = 1;
+    p.pf_prefix = reinterpret_cast<int32_t*>(static_cast<char*>(workspace) + wl.pf_prefix_off);
+    p.pf_o = reinterpret_cast<float*>(static_cast<char*>(workspace) + wl.pf_o_off);
+    p.pf_lse = reinterpret_cast<float*>(static_cast<char*>(workspace) + wl.pf_lse_off);
+    p.grid = wl.pf_grid;
     // K/V boxes are 64 columns wide (128 bytes) to match the 128-byte swizzle
     // of the MMA tiles.
     const int32_t gh = prefill_heads_per_tile(group);
@@ -557,6 +588,7 @@ pa_status pa_attention_cascade(const void* q, const void* k_cache, const void* v
   a.grid = 0;
   a.hpu = 1;
   a.scale_log2 = scale_log2;
+  a.wait_limit_ns = wait_limit_ns();
   a.skip_blocks = num_groups > 0 ? shared_blocks : nullptr;
   a.l1_o = reinterpret_cast<float*>(ws + wl.l1_o_off);
   a.l1_lse = reinterpret_cast<float*>(ws + wl.l1_lse_off);
@@ -586,6 +618,7 @@ pa_status pa_attention_cascade(const void* q, const void* k_cache, const void* v
     p.max_query_len = max_group_size;
     p.num_q_tokens = num_seqs;
     p.scale_log2 = scale_log2;
+    p.wait_limit_ns = wait_limit_ns();
     p.groups = groups;
     p.skip_blocks = shared_blocks;
     p.num_groups = num_groups;
@@ -593,6 +626,10 @@ pa_status pa_attention_cascade(const void* q, const void* k_cache, const void* v
     p.l1_lse = reinterpret_cast<float*>(ws + wl.l1_lse_off);
     p.l1_max_chunks = max_chunks;
     p.l1_chunk_blocks = chunk_blocks;
+    p.pf_prefix = nullptr;
+    p.pf_o = nullptr;
+    p.pf_lse = nullptr;
+    p.grid = 0;
     const int32_t gh = prefill_heads_per_tile(num_q_heads / cache->num_kv_heads);
     const uint64_t qd[3] = {uint64_t(cache->head_dim), uint64_t(num_q_heads), uint64_t(num_seqs)};
     const uint64_t qs[2] = {uint64_t(cache->head_dim) * 2, uint64_t(num_q_heads) * cache->head_dim * 2};
@@ -608,6 +645,10 @@ pa_status pa_attention_cascade(const void* q, const void* k_cache, const void* v
   e = launch_decode_combine(a, *cache, s);
   if (e != cudaSuccess) return cuda_fail(e, "decode combine launch");
   return PA_OK;
+}
+
+uint64_t pa_set_wait_limit_ns(uint64_t limit_ns) {
+  return g_wait_limit_ns.exchange(limit_ns, std::memory_order_relaxed);
 }
 
 pa_status pa_get_debug_status(void* stream, int32_t* host_flag) {

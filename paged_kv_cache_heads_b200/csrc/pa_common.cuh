@@ -2,9 +2,10 @@
 //
 // PTX wrappers for mbarriers, TMA tensor loads, bounded waits and the
 // library's device status word. Every wait in this library is bounded: when a
-// barrier does not complete within PA_WAIT_LIMIT_NS the waiting thread sets
-// PA_FLAG_WAIT_TIMEOUT in the status word and the kernel abandons its work,
-// so a logic error reports itself instead of hanging the GPU.
+// barrier does not complete within the call's limit (pa_set_wait_limit_ns,
+// default PA_WAIT_LIMIT_NS = 2 s) the waiting thread sets PA_FLAG_WAIT_TIMEOUT
+// in the status word and the kernel abandons its work, so a logic error
+// reports itself instead of hanging the GPU.
 #pragma once
 
 #include <cuda.h>
@@ -13,10 +14,7 @@
 #include <stdint.h>
 
 #include "pa.h"
-
-#ifndef PA_WAIT_LIMIT_NS
-#define PA_WAIT_LIMIT_NS 2000000000ull   // 2 s per wait
-#endif
+#include "pa_internal.h"
 
 namespace pa {
 
@@ -92,21 +90,40 @@ __device__ __forceinline__ bool mbar_test_wait(uint64_t* bar, uint32_t parity) {
 }
 
 // Wait until the phase with the given parity has completed. Returns false
-// (after raising PA_FLAG_WAIT_TIMEOUT) when the wait exceeds the limit or
-// another thread of the grid has already reported a timeout.
-__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, unsigned* status) {
+// (after raising PA_FLAG_WAIT_TIMEOUT) when the wait exceeds `limit_ns` or
+// another thread of the grid has already reported a timeout. The limit is
+// checked after the second failed poll (so a limit of 0 gives up on any wait
+// that is not already satisfied) and then every 1024 polls.
+__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, unsigned* status,
+                                          uint64_t limit_ns = PA_WAIT_LIMIT_NS) {
   if (mbar_try_wait(bar, parity)) return true;
   const uint64_t t0 = globaltimer_ns();
-  uint32_t spins = 0;
-  while (!mbar_try_wait(bar, parity)) {
-    if ((++spins & 1023u) == 0) {
-      if (globaltimer_ns() - t0 > PA_WAIT_LIMIT_NS || flag_raised(status, PA_FLAG_WAIT_TIMEOUT)) {
-        raise_flag(status, PA_FLAG_WAIT_TIMEOUT);
-        return false;
-      }
+  for (uint32_t spins = 1;; ++spins) {
+    if (mbar_try_wait(bar, parity)) return true;
+    const bool check = spins == 1 || (spins & 1023u) == 0;
+    if (check && (globaltimer_ns() - t0 >= limit_ns ||
+                  ((spins & 1023u) == 0 && flag_raised(status, PA_FLAG_WAIT_TIMEOUT)))) {
+      raise_flag(status, PA_FLAG_WAIT_TIMEOUT);
+      return false;
     }
   }
-  return true;
+}
+
+// Drain wait: used before a CTA exits, for copies or MMAs it issued itself,
+// which the hardware completes by itself. Always the default bound, whatever
+// limit the call runs with and whether or not a timeout was raised elsewhere,
+// so that nothing is still writing into this CTA's shared memory (or TMEM)
+// when it exits.
+__device__ __forceinline__ bool mbar_drain(uint64_t* bar, uint32_t parity, unsigned* status) {
+  if (mbar_try_wait(bar, parity)) return true;
+  const uint64_t t0 = globaltimer_ns();
+  for (uint32_t spins = 1;; ++spins) {
+    if (mbar_try_wait(bar, parity)) return true;
+    if ((spins & 1023u) == 0 && globaltimer_ns() - t0 >= PA_WAIT_LIMIT_NS) {
+      raise_flag(status, PA_FLAG_WAIT_TIMEOUT);
+      return false;
+    }
+  }
 }
 
 // ---------------------------------------------------------------- TMA

@@ -9,6 +9,10 @@
 
 #include "pa.h"
 
+#ifndef PA_WAIT_LIMIT_NS
+#define PA_WAIT_LIMIT_NS 2000000000ull  // default bound of a device-side wait: 2 s
+#endif
+
 namespace pa {
 
 // Device-side work description of one pa_attention call (decode part).
@@ -31,6 +35,7 @@ struct DecodeArgs {
   int32_t grid;         // CTAs of the decode grid (set by the decode launcher)
   int32_t hpu;          // query heads per unit of the decode grid (set by the decode launcher)
   float scale_log2;     // scale * log2(e)
+  uint64_t wait_limit_ns;  // bound of every device-side wait on another party (pa_set_wait_limit_ns)
   // Cascade (shared-prefix) decode; all null / 0 otherwise.
   const int32_t* skip_blocks;  // [num_seqs] leading table blocks read by the prefix pass instead
   const float* l1_o;           // [num_seqs * num_q_heads * l1_max_chunks][head_dim] prefix-pass partials
@@ -54,6 +59,7 @@ struct PrefillArgs {
   int32_t max_query_len;
   int32_t num_q_tokens;
   float scale_log2;
+  uint64_t wait_limit_ns;  // bound of every device-side wait on another party (pa_set_wait_limit_ns)
   // Cascade prefix pass (kernel instantiated with the cascade flag): work
   // items run over the groups' shared blocks instead of the prefill rows.
   const int32_t* groups;       // [num_groups][2]: first member sequence, member count
@@ -63,10 +69,27 @@ struct PrefillArgs {
   float* l1_lse;
   int32_t l1_max_chunks;
   int32_t l1_chunk_blocks;
+  // Prefill rows (workspace): key tiles before each sequence, then the grid
+  // the tiles were split over and their total ([num_seqs + 3], written by the
+  // kernel for the merge); partials of split work items, two slots per CTA of
+  // 256 rows each ([2 * grid][256][head_dim] and [2 * grid][256]).
+  int32_t* pf_prefix;
+  float* pf_o;
+  float* pf_lse;
+  int32_t grid;                // CTAs of the prefill grid (prefill_grid)
 };
+
+// CTAs of the prefill grid for a call with these host bounds: one per SM,
+// fewer when the call cannot have 8 key tiles of work per CTA. The workspace
+// holds two partial slots per CTA.
+int32_t prefill_grid(int32_t num_seqs, int32_t num_q_heads, int32_t num_kv_heads, int32_t max_query_len,
+                     int32_t max_context_len);
 
 // Sets the calling thread's pa_last_error() message.
 void set_last_error(const char* msg);
+
+// Current bound of the kernels' device-side waits (pa_set_wait_limit_ns).
+uint64_t wait_limit_ns();
 
 // Upper bound on the decode grid; the workspace holds S*Hq/GH + this many partial slots.
 int32_t decode_max_grid();
