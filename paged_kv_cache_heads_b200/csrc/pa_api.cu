@@ -445,6 +445,8 @@ pa_status pa_attention(const void* q, const void* k_cache, const void* v_cache,
   if (e != cudaSuccess) return cuda_fail(e, "decode combine launch");
   if (max_query_len > 1) {
     PrefillArgs p;
+    p.k_cache = k_cache;
+    p.v_cache = v_cache;
     p.out = out;
     p.block_tables = block_tables;
     p.context_lens = context_lens;
@@ -604,6 +606,8 @@ pa_status pa_attention_cascade(const void* q, const void* k_cache, const void* v
   // 2. each group's shared blocks, read once for all its members: partials
   if (num_groups > 0) {
     PrefillArgs p;
+    p.k_cache = k_cache;
+    p.v_cache = v_cache;
     p.out = out;
     p.block_tables = block_tables;
     p.context_lens = context_lens;

@@ -45,6 +45,8 @@ struct DecodeArgs {
 };
 
 struct PrefillArgs {
+  const void* k_cache;  // [num_blocks][block_size][num_kv_heads][head_dim]
+  const void* v_cache;
   void* out;
   const int32_t* block_tables;
   const int32_t* context_lens;

@@ -12,30 +12,36 @@
 //  * A Q tile is 128 query rows: 128/GH tokens x the GH query heads of one GQA
 //    group, so each gathered K/V tile serves every head of the group. A work
 //    item (pair) is two consecutive Q tiles of one sequence and head group:
-//    both tiles multiply the same K/V tiles, which halves the shared-memory
-//    traffic per MMA and gives the tensor pipe two independent chains.
-//  * Keys come in tiles of 64. Every pair's key tiles are numbered
-//    contiguously (sequence, head group, pair) and the grid splits the whole
-//    range evenly (stream-K): CTA c takes tiles [c*T/G, (c+1)*T/G), so long
-//    and short pairs balance. A pair one CTA covers entirely is written
-//    straight to the output; otherwise each covering CTA leaves a partial
+//    both multiply the same K/V tiles, and their two dependency chains keep
+//    the tensor pipe busy while either one's softmax runs (ping-pong).
+//  * Keys come in tiles of 128: an M=128, N=128, K=16 MMA keeps the tensor
+//    pipe above 90% busy where N=64 reaches about 55% (measured).
+//  * Work units: a pair's key tiles plus a fixed number of units for the cost
+//    of starting and finishing it (Q tiles, epilogue, pipeline refill); all
+//    units are numbered contiguously (sequence, head group, pair) and the grid
+//    splits the whole range evenly (stream-K): CTA c takes units
+//    [c*T/G, (c+1)*T/G). A pair one CTA covers entirely is written straight to
+//    the output; otherwise each covering CTA leaves a partial
 //    (O / l, m + log2 l) per row and prefill_combine_kernel merges them.
-//  * Warp 9 (producer) loads both Q tiles per segment and, per key tile, each
-//    KV block of the tile with TMA (box {64, 1, bs, 1}, 128-byte swizzle) into
-//    a ring of K/V stages.
-//  * Warp 8 (one thread) issues S_i = Q_i K^T (M=128, N=64) into the TMEM
-//    columns of Q tile i as soon as its softmax warps have loaded the previous
-//    S into registers, so the next scores are computed during the current
-//    softmax; and O_i += P_i V with P_i read from tensor memory (M=128,
-//    N=head_dim). No MMA waits for another MMA: the tensor pipe stays fed.
-//    tcgen05.commit arrives on mbarriers; every wait is bounded.
+//  * Warp 9 loads both Q tiles of a segment with TMA. Warps 9 and 10 gather
+//    each key tile's K and V rows through the block table with 16-byte
+//    cp.async copies straight into the 128-byte swizzled layout of the MMA
+//    operands (a tensor-copy box per KV block and 64 columns would cost one
+//    serialised issue each), into a ring of K/V stages. Rows at or beyond L
+//    (the unfilled tail of the last block, blocks past the sequence) are
+//    filled with zeros, so stale bits there cannot reach the output.
+//  * TMEM (512 columns): S_i of Q tile i in columns [128 i, 128 i + 128);
+//    its softmax writes P_i as bf16 over the first 64 of them; O_i at
+//    256 + i * head_dim. Warp 8 (one thread) issues, per key tile j:
+//    O_0 += P_0(j-1) V(j-1), S_0(j) = Q_0 K(j)^T, then the same for tile 1.
+//    The MMAs of one thread run in issue order, so S_i(j) overwrites P_i(j-1)
+//    only after the product that reads it, and a completed S_i(j) implies a
+//    completed O_i update for j-1. tcgen05.commit arrives on mbarriers; every
+//    wait is bounded.
 //  * Warps 0-3 and 4-7 run the softmax of Q tile 0 and 1: one row per thread
 //    (TMEM lane = row), fp32 online softmax with exp2 on the scale folded into
-//    log2 e, P written as bf16 into one of two TMEM P buffers of the tile (the
-//    MMA reads it there). O is rescaled in TMEM only when a row's running max
-//    grows by more than 2^8.
-//  * V rows at or beyond L inside the last key tile hold stale bits; the MMA
-//    warp zeroes them before the P.V product, so they cannot reach the output.
+//    log2 e. O is rescaled in TMEM only when a row's running max grows by
+//    more than 2^8.
 #include <math_constants.h>
 
 #include "decode_common.cuh"
@@ -46,10 +52,20 @@
 namespace pa {
 namespace {
 
-constexpr int kBN = 64;             // keys per tile
+constexpr int kBN = 128;            // keys per tile
 constexpr float kRescaleLog2 = 8.f;
 constexpr int kMinTilesPerCta = 8;  // a CTA gets at least this many key tiles of work
-constexpr int kThreads = 320;       // softmax warps 0-7, MMA warp 8, producer warp 9
+// Work units: a pair's key tiles plus this many units of fixed cost for its
+// segment (loading its Q tiles, the epilogue, refilling the pipeline), so that
+// a CTA whose range crosses many short pairs is given fewer key tiles.
+constexpr int kSegUnits = 2;
+// Warps 0-7 softmax, 8 MMA issue, 9-10 K producers, 11-12 V producers, 13-15
+// idle. Warpgroups 2-3 (warps 8-15) hand registers to warpgroups 0-1:
+// 8 * 32 * kRegSoftmax + 8 * 32 * kRegOther = 512 threads * 128 registers.
+constexpr int kThreads = 512;
+constexpr int kRegSoftmax = 184;
+constexpr int kRegOther = 72;
+static_assert(8 * 32 * kRegSoftmax + 8 * 32 * kRegOther == kThreads * 128, "register split must match the launch");
 constexpr int kMmaWarp = 8;
 constexpr int kLoadWarp = 9;
 
@@ -60,25 +76,34 @@ struct PrefillCfg {
   static constexpr int kHalves = D / 64;     // 128-byte column groups
   static constexpr int kQTileB = 128 * D * 2;
   static constexpr int kKB = kBN * D * 2;    // one K (or V) tile
-  static constexpr int kStageB = 2 * kKB;
-  static constexpr int kNST = D == 128 ? 4 : 6;  // K/V stages
+  // K and V tiles take turns in a ring of slots: K(j) in slot 2j, V(j) in slot
+  // 2j + 1 (mod kNSL). A K slot is free again once S(j) is done, a V slot once
+  // O += P V(j) is, so the next loads start as early as each allows.
+  static constexpr int kNSL = D == 128 ? 4 : 8;
   static constexpr int kBlk = kBN / BS;          // KV blocks per key tile
+  static constexpr int kCPR = D / 8;             // 16-byte chunks per key row
+  static constexpr int kRPS = 64 / kCPR;  // rows a pair of producer warps copies per step
   static constexpr int kStageOff = 2 * kQTileB;
-  static constexpr int kBarOff = kStageOff + kNST * kStageB;
-  // q_full, q_empty, mma_done, kv_full[NST], kv_empty[NST], s_full[2], s_free[2], p_full[4], pv_done[4]
-  static constexpr int kNumBars = 3 + 2 * kNST + 12;
+  static constexpr int kBarOff = kStageOff + kNSL * kKB;
+  // q_full, q_empty, mma_done, kv_full[NSL], kv_empty[NSL], s_full[2], p_full[2], pv_done[2]
+  static constexpr int kNumBars = 3 + 2 * kNSL + 6;
   static constexpr int kTmemOff = kBarOff + kNumBars * 8;
   static constexpr int kScanOff = (kTmemOff + 16 + 15) / 16 * 16;
   static constexpr int kSeqOff = kScanOff + 32 * 4;
-  // TMEM columns: S of Q tile i at 64 i; its P buffers b at 128 + 64 i + 32 b
-  // (64 bf16 keys packed two per column); O of Q tile i at 256 + i * D.
   static constexpr uint32_t kTmemCols = 512;
-  static constexpr uint32_t kPCol = 128;
   static constexpr uint32_t kOCol = 256;
   static constexpr uint32_t kIdescS = tc::idesc_bf16_f32(128, kBN, 0, 0);
   static constexpr uint32_t kIdescO = tc::idesc_bf16_f32(128, D, 0, 1);
   static size_t smem_bytes(int num_seqs) { return 1024 + kSeqOff + 4ull * (num_seqs + 1); }
 };
+
+// 2^x with the hardware's approximate exp2 (denormal results flush to zero,
+// 2^-inf = 0): the probabilities are rounded to bf16 right after.
+__device__ __forceinline__ float ex2_ftz(float x) {
+  float y;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
 
 // Key tiles a pair (or its first Q tile) needs: through the last visible key
 // of its last row, tok_end being one past that row's token.
@@ -92,10 +117,15 @@ struct PSeg {
   int nt, nt0;       // key tiles of the pair, of its first Q tile
   int slot;          // -1: this CTA covers the whole pair; else its partial slot
   bool t1;           // the second Q tile holds at least one row of the sequence
+  int adv;           // work units from the segment's start to the next segment
+  int64_t tile0;     // unit of the pair's first key tile
 };
 
-// The segment of CTA `cta` (tile range [beg, end)) that starts at global key
-// tile b. prefix[s] = key tiles before sequence s (prefix[num_seqs] > b).
+// The segment of CTA `cta` (unit range [beg, end)) that starts at unit b.
+// prefix[s] = work units before sequence s (prefix[num_seqs] > b). A pair of
+// nt key tiles occupies kSegUnits + nt units: its fixed cost, then one unit per
+// key tile. The segment holds key tiles [j_lo, j_hi) of the pair (possibly none,
+// when b and end fall in the fixed-cost units); adv units lead to the next one.
 template <int GH>
 __device__ __forceinline__ void locate(int64_t b, int64_t beg, int64_t end, int cta, const int* prefix,
                                        int num_seqs, int HGp, const PrefillArgs& a, PSeg& g) {
@@ -109,25 +139,32 @@ __device__ __forceinline__ void locate(int64_t b, int64_t beg, int64_t end, int 
   g.L = __ldg(a.context_lens + lo);
   g.r0 = __ldg(a.query_start_loc + lo);
   g.ql = __ldg(a.query_start_loc + lo + 1) - g.r0;
-  const int tiles_hg = (prefix[lo + 1] - prefix[lo]) / HGp;
+  const int units_hg = (prefix[lo + 1] - prefix[lo]) / HGp;
   int off = static_cast<int>(b - prefix[lo]);
-  g.hg = off / tiles_hg;
-  off -= g.hg * tiles_hg;
+  g.hg = off / units_hg;
+  off -= g.hg * units_hg;
   int pt = 0, nt;
+  int64_t u0 = prefix[lo] + static_cast<int64_t>(g.hg) * units_hg;  // the pair's first unit
   for (;;) {
     nt = tiles_through(g.L, g.ql, min((pt + 1) * PT, g.ql));
-    if (off < nt) break;
-    off -= nt;
+    if (off < kSegUnits + nt) break;
+    off -= kSegUnits + nt;
+    u0 += kSegUnits + nt;
     ++pt;
   }
   g.pt = pt;
   g.nt = nt;
   g.nt0 = tiles_through(g.L, g.ql, min(pt * PT + TOK, g.ql));
   g.t1 = pt * PT + TOK < g.ql;
-  g.j_lo = off;
-  const int64_t room = end - b;
-  g.j_hi = off + static_cast<int>(room < nt - off ? room : nt - off);
-  g.slot = (off == 0 && g.j_hi == nt) ? -1 : 2 * cta + (b > beg ? 1 : 0);
+  g.tile0 = u0 + kSegUnits;
+  const int64_t jl = b - g.tile0, jh = end - g.tile0;
+  g.j_lo = static_cast<int>(jl > 0 ? jl : 0);
+  g.j_hi = static_cast<int>(jh < nt ? (jh > 0 ? jh : 0) : nt);
+  const int64_t pair_end = g.tile0 + nt;
+  g.adv = static_cast<int>((pair_end < end ? pair_end : end) - b);
+  // a split pair's first piece (its tiles start in this CTA) takes slot 2 cta + 1,
+  // a later piece (the pair began in an earlier CTA) slot 2 cta
+  g.slot = (g.j_lo == 0 && g.j_hi == nt) ? -1 : 2 * cta + (g.j_lo == 0 ? 1 : 0);
 }
 
 template <int D, int BS, int GH>
@@ -135,19 +172,18 @@ __global__ void __launch_bounds__(kThreads, 1)
     paged_prefill_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constant__ CUtensorMap kmap,
                          const __grid_constant__ CUtensorMap vmap, const PrefillArgs a) {
   using C = PrefillCfg<D, BS, GH>;
-  constexpr int NST = C::kNST;
+  constexpr int NSL = C::kNSL;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::kBarOff);
   uint64_t* q_full = bars + 0;
   uint64_t* q_empty = bars + 1;
   uint64_t* mma_done = bars + 2;
-  uint64_t* kv_full = bars + 3;     // [NST]
-  uint64_t* kv_empty = kv_full + NST;
-  uint64_t* s_full = kv_empty + NST;  // [Q tile]: S computed
-  uint64_t* s_free = s_full + 2;      // [Q tile]: S loaded into registers by the softmax warps
-  uint64_t* p_full = s_free + 2;      // [Q tile * 2 + P buffer]
-  uint64_t* pv_done = p_full + 4;     // [Q tile * 2 + P buffer]
+  uint64_t* kv_full = bars + 3;     // [NSL]: slot loaded
+  uint64_t* kv_empty = kv_full + NSL;  // [NSL]: slot consumed
+  uint64_t* s_full = kv_empty + NSL;  // [Q tile]: S computed (and every earlier MMA)
+  uint64_t* p_full = s_full + 2;      // [Q tile]: P written (and O rescaled) by its softmax warps
+  uint64_t* pv_done = p_full + 2;     // [Q tile]: O += P V done
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + C::kTmemOff);
   int* warp_tot = reinterpret_cast<int*>(smem + C::kScanOff);
   int* prefix = reinterpret_cast<int*>(smem + C::kSeqOff);
@@ -161,25 +197,18 @@ __global__ void __launch_bounds__(kThreads, 1)
     mbar_init(q_full, 1);
     mbar_init(q_empty, 1);
     mbar_init(mma_done, 1);
-    for (int i = 0; i < NST; ++i) {
-      mbar_init(&kv_full[i], 1);
+    for (int i = 0; i < NSL; ++i) {
+      mbar_init(&kv_full[i], 64);  // one arrival per lane of the producer pair that fills it
       mbar_init(&kv_empty[i], 1);
     }
     for (int i = 0; i < 2; ++i) {
       mbar_init(&s_full[i], 1);
-      mbar_init(&s_free[i], 4);  // one arrival per softmax warp of the Q tile
-    }
-    for (int i = 0; i < 4; ++i) {
-      mbar_init(&p_full[i], 4);
+      mbar_init(&p_full[i], 4);  // one arrival per softmax warp of the Q tile
       mbar_init(&pv_done[i], 1);
     }
     fence_barrier_init();
   }
-  if (warp == kLoadWarp && lane == 0) {
-    tma_prefetch_desc(&qmap);
-    tma_prefetch_desc(&kmap);
-    tma_prefetch_desc(&vmap);
-  }
+  if (warp >= kLoadWarp && lane == 0) tma_prefetch_desc(&qmap);
 
   // ---- key tiles of every prefill sequence, and their prefix. This grid is
   // chained after the decode merge; every input it reads was complete before
@@ -198,7 +227,8 @@ __global__ void __launch_bounds__(kThreads, 1)
             r0 + ql > a.num_q_tokens) {
           raise_flag(a.status, PA_FLAG_CONTEXT_RANGE);
         } else {
-          for (int pt = 0; pt * C::kPairTok < ql; ++pt) n += tiles_through(L, ql, min((pt + 1) * C::kPairTok, ql));
+          for (int pt = 0; pt * C::kPairTok < ql; ++pt)
+            n += kSegUnits + tiles_through(L, ql, min((pt + 1) * C::kPairTok, ql));
           n *= HGp;
         }
       }
@@ -235,169 +265,196 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int64_t end = static_cast<int64_t>(blockIdx.x + 1) * T / Geff;
   const int cta = static_cast<int>(blockIdx.x);
 
-  if (warp == kLoadWarp) {
-    // ================= producer: Q tiles per segment, K/V blocks per key tile
+  // Registers move from warpgroups 2-3 (MMA issue, producers, idle) to the
+  // softmax warpgroups: each role calls setmaxnreg first thing.
+  if (warp >= kLoadWarp + 4) {
+    setmaxnreg_dec<kRegOther>();  // idle warps only hand over their registers
+  } else if (warp >= kLoadWarp) {
+    setmaxnreg_dec<kRegOther>();
+    // ================= producers. Warps kLoadWarp, +1 gather every key tile's K,
+    // warps kLoadWarp + 2, +3 its V, each pair half of the rows (so each ring
+    // slot is filled by one pair, in order), with 16-byte cp.async copies into the 128-byte swizzled layout
+    // the MMAs read (chunk c of row r at r * 128 + ((c ^ (r & 7)) << 4) within
+    // its 64-column half); rows at or beyond L are filled with zeros, so stale
+    // bits in the unfilled tail of the last block never reach the MMAs. Every
+    // lane arrives on kv_full asynchronously, when its copies have landed; the
+    // MMA thread fences them for the tensor cores. The K warp also loads each
+    // segment's two Q tiles (TMA), after the segment's first K tile: the Q
+    // buffer frees only when the previous segment's last scores are done.
+    const int kv = (warp - kLoadWarp) >> 1;                 // 0: K, 1: V
+    const int p = ((warp - kLoadWarp) & 1) * 32 + lane;  // thread of the pair
+    const int ch = p % C::kCPR;  // 16-byte chunk of a row
+    const int rg = p / C::kCPR;  // first row of this thread; rows rg + kRPS i
+    const uint32_t dst_col = (ch >> 3) * (kBN * 128) + rg * 128;
+    const int64_t tok_bytes = static_cast<int64_t>(a.num_kv_heads) * D * 2;
     bool ok = true;
-    uint32_t kt = 0, nq = 0;  // key tiles and Q loads issued
+    uint32_t kt = 0, nq = 0;  // key tiles and segments of this CTA so far
+    uint32_t my_q = 0;        // 1 + the segment of the last Q load this warp issued (0: none)
     for (int64_t b = beg; b < end && ok;) {
       PSeg g;
       locate<GH>(b, beg, end, cta, prefix, S, HGp, a, g);
-      b += g.j_hi - g.j_lo;
+      b += g.adv;
+      if (g.j_lo == g.j_hi) continue;  // only fixed-cost units of a pair
       const int hq0 = g.hg * GH, hk = hq0 / G;
-      const int t0 = g.pt * C::kPairTok;
-      if (lane == 0) {
-        ok = mbar_wait(q_empty, (nq & 1) ^ 1, a.status, a.wait_limit_ns);
-        if (ok) {
-          mbar_arrive_expect_tx(q_full, 2 * C::kQTileB);
-#pragma unroll
-          for (int qi = 0; qi < 2; ++qi)
-#pragma unroll
-            for (int h = 0; h < C::kHalves; ++h)
-              tma_load_3d(smem + qi * C::kQTileB + h * 128 * 128, &qmap, q_full, h * 64, hq0,
-                          g.r0 + t0 + qi * C::kTOK);
-        }
-      }
-      ok = __shfl_sync(0xffffffffu, ok, 0) != 0;
-      if (!ok) break;
-      ++nq;
       const int* row = a.block_tables + static_cast<size_t>(g.s) * a.max_blocks_per_seq;
       const int nblk_valid = (g.L + BS - 1) / BS;
-      for (int j = g.j_lo; j < g.j_hi; ++j, ++kt) {
-        const uint32_t st = kt % NST;
-        if (lane == 0) {
-          ok = mbar_wait(&kv_empty[st], ((kt / NST) & 1) ^ 1, a.status, a.wait_limit_ns);
-          if (ok) mbar_arrive_expect_tx(&kv_full[st], C::kStageB);
-        }
-        ok = __shfl_sync(0xffffffffu, ok, 0) != 0;
-        if (!ok) break;
-        if (lane < C::kBlk) {
-          const int lb = j * C::kBlk + lane;
-          int phys = -1;  // a block past the sequence: an out-of-range box, filled with zeros
-          if (lb < nblk_valid) {
-            phys = __ldg(row + lb);
-            if (phys < 0 || phys >= a.num_blocks) {
-              raise_flag(a.status, PA_FLAG_BLOCK_RANGE);
-              phys = -1;
-            }
-          }
-          uint8_t* ks = smem + C::kStageOff + st * C::kStageB;
-          uint8_t* vs = ks + C::kKB;
+      const char* kcol = static_cast<const char*>(a.k_cache) + static_cast<size_t>(hk) * D * 2 + ch * 16;
+      const char* vcol = static_cast<const char*>(a.v_cache) + static_cast<size_t>(hk) * D * 2 + ch * 16;
+      for (int j = g.j_lo; j < g.j_hi && ok; ++j, ++kt) {
+        // byte offset of this lane's first row (rg) in each block of the tile;
+        // -1: the block is past the sequence (or invalid) and its rows are zero-filled
+        int64_t boff[C::kBlk];
 #pragma unroll
-          for (int h = 0; h < C::kHalves; ++h) {
-            tma_load_4d(ks + h * kBN * 128 + lane * BS * 128, &kmap, &kv_full[st], h * 64, hk, 0, phys);
-            tma_load_4d(vs + h * kBN * 128 + lane * BS * 128, &vmap, &kv_full[st], h * 64, hk, 0, phys);
+        for (int bb = 0; bb < C::kBlk; ++bb) {
+          const int lb = j * C::kBlk + bb;
+          boff[bb] = -1;
+          if (lb < nblk_valid) {
+            const int pb = __ldg(row + lb);
+            if (pb >= 0 && pb < a.num_blocks) boff[bb] = (static_cast<int64_t>(pb) * BS + rg) * tok_bytes;
+            else if (p == 0) raise_flag(a.status, PA_FLAG_BLOCK_RANGE);
+          }
+        }
+        const int kbase = j * kBN;
+        const bool full = kbase + kBN <= g.L;  // every row of the tile is a live key
+        {
+          const uint32_t n = 2 * kt + kv, sl = n % NSL;
+          if (lane == 0) ok = mbar_wait(&kv_empty[sl], ((n / NSL) & 1) ^ 1, a.status, a.wait_limit_ns);
+          ok = __shfl_sync(0xffffffffu, ok, 0) != 0;
+          if (!ok) break;
+          const uint32_t dst = smem_u32(smem + C::kStageOff + sl * C::kKB) + dst_col;
+          const char* src = kv ? vcol : kcol;
+#pragma unroll
+          for (int i = 0; i < kBN / C::kRPS; ++i) {
+            const int r = rg + C::kRPS * i;
+            // rg < kRPS <= BS, so the block and the row's offset in it are known at compile time
+            const int64_t bo = boff[(C::kRPS * i) / BS];
+            const bool live = bo >= 0 && (full || kbase + r < g.L);
+            const int64_t off = bo + static_cast<int64_t>((C::kRPS * i) % BS) * tok_bytes;
+            cp_async16(dst + C::kRPS * i * 128 + (((ch & 7) ^ (r & 7)) << 4), src + (live ? off : 0),
+                       live ? 16u : 0u);
+          }
+          cp_async_arrive(&kv_full[sl]);
+          if (warp == kLoadWarp && j == g.j_lo) {  // this segment's Q tiles
+            if (lane == 0) {
+              ok = mbar_wait(q_empty, (nq & 1) ^ 1, a.status, a.wait_limit_ns);
+              if (ok) {
+                mbar_arrive_expect_tx(q_full, 2 * C::kQTileB);
+#pragma unroll
+                for (int qi = 0; qi < 2; ++qi)
+#pragma unroll
+                  for (int h = 0; h < C::kHalves; ++h)
+                    tma_load_3d(smem + qi * C::kQTileB + h * 128 * 128, &qmap, q_full, h * 64, hq0,
+                                g.r0 + g.pt * C::kPairTok + qi * C::kTOK);
+              }
+            }
+            ok = __shfl_sync(0xffffffffu, ok, 0) != 0;
+            if (!ok) break;
+            my_q = nq + 1;
           }
         }
       }
+      ++nq;
     }
-    // Before the CTA exits no copy may still be landing in its shared memory:
-    // the last load of every stage and the last Q load (default bound).
-    if (lane == 0) {
-      for (uint32_t i = kt > static_cast<uint32_t>(NST) ? kt - NST : 0; i < kt; ++i)
-        mbar_drain(&kv_full[i % NST], (i / NST) & 1, a.status);
-      if (nq > 0) mbar_drain(q_full, (nq - 1) & 1, a.status);
-    }
+    // every copy of this thread has landed before the CTA exits
+    cp_async_wait_all();
+    // the last Q load this warp issued (default bound): one Q load is in flight
+    // at a time, since each waits for the previous segment's scores
+    if (lane == 0 && my_q > 0) mbar_drain(q_full, (my_q - 1) & 1, a.status);
     __syncwarp();
   } else if (warp == kMmaWarp) {
-    // ================= MMA issue (lane 0; the whole warp zeroes stale V rows)
-    // Per key tile: S of both Q tiles (once their softmax warps hold the
-    // previous S in registers), then the P.V products of the previous tile
-    // once the softmax warps have written its P. The tensor pipe thus always
-    // holds the next scores while the softmax of the current ones runs.
+    setmaxnreg_dec<kRegOther>();
+    // ================= MMA issue (lane 0). Per key tile j, for Q tile 0 then 1:
+    // O_i += P_i(j-1) V(j-1) once its softmax warps have written P_i(j-1), then
+    // S_i(j) = Q_i K(j)^T into the same TMEM columns. The softmax of one Q
+    // tile thus runs while the tensor pipe works on the other.
     bool ok = true;
     uint32_t kt = 0, nq = 0;
-    uint32_t cnt[2] = {0, 0};  // S / P.V products issued per Q tile
+    uint32_t ns[2] = {0, 0};  // S products issued per Q tile (= P tiles to consume)
     auto wait1 = [&](uint64_t* bar, uint32_t parity) {
       bool r = true;
       if (lane == 0) r = mbar_wait(bar, parity, a.status, a.wait_limit_ns);
       return __shfl_sync(0xffffffffu, r, 0) != 0;
     };
-    // O_i += P_i V for the tile in stage st whose products are numbered c[i]
-    auto issue_pv = [&](uint32_t st, const bool* act, const uint32_t* c, bool* first) {
+    // O_qi += P_qi V for the V tile in slot sl, whose P is S product number c of Q tile qi
+    auto issue_pv = [&](int qi, uint32_t sl, uint32_t c, bool accumulate) {
+      if (!wait1(&p_full[qi], c & 1)) return false;
+      if (lane == 0) {
+        tc::fence_after_sync();
+        const uint32_t v_addr = smem_u32(smem + C::kStageOff + sl * C::kKB);
+        const uint32_t p_t = tmem + qi * 128;
 #pragma unroll
-      for (int qi = 0; qi < 2; ++qi) {
-        if (!act[qi]) continue;
-        const uint32_t bb = c[qi] & 1;
-        if (!wait1(&p_full[qi * 2 + bb], (c[qi] >> 1) & 1)) return false;
-        if (lane == 0) {
-          tc::fence_after_sync();
-          const uint32_t v_addr = smem_u32(smem + C::kStageOff + st * C::kStageB + C::kKB);
-          const uint32_t p_t = tmem + C::kPCol + qi * 64 + bb * 32;
-#pragma unroll
-          for (int kk = 0; kk < kBN / 16; ++kk)
-            tc::mma_bf16_ta(tmem + C::kOCol + qi * D, p_t + kk * 8,
-                            tc::sw128_desc(v_addr + kk * 16 * 128, kBN * 128, 1024), C::kIdescO,
-                            !first[qi] || kk > 0);
-          tc::commit(&pv_done[qi * 2 + bb]);
-        }
-        first[qi] = false;
+        for (int kk = 0; kk < kBN / 16; ++kk)
+          tc::mma_bf16_ta(tmem + C::kOCol + qi * D, p_t + kk * 8,
+                          tc::sw128_desc(v_addr + kk * 16 * 128, kBN * 128, 1024), C::kIdescO,
+                          accumulate || kk > 0);
+        tc::commit(&pv_done[qi]);
       }
-      if (lane == 0) tc::commit(&kv_empty[st]);
       return true;
     };
     for (int64_t b = beg; b < end && ok;) {
       PSeg g;
       locate<GH>(b, beg, end, cta, prefix, S, HGp, a, g);
-      b += g.j_hi - g.j_lo;
+      b += g.adv;
+      if (g.j_lo == g.j_hi) continue;  // only fixed-cost units of a pair
       if (!(ok = wait1(q_full, nq & 1))) break;
       ++nq;
       const uint32_t q_addr = smem_u32(smem);
-      bool first[2] = {true, true};
-      bool pact[2] = {false, false};
-      uint32_t pc[2] = {0, 0}, pst = 0;
-      bool have_prev = false;
+      bool pact[2] = {false, false};     // Q tile active in the previous key tile
+      bool acc[2] = {false, false};      // O_i already holds a product of this segment
+      uint32_t pc[2] = {0, 0}, pvs = 0;  // its S number, and the previous tile's V slot
       for (int j = g.j_lo; j < g.j_hi; ++j, ++kt) {
-        const uint32_t st = kt % NST;
-        if (!(ok = wait1(&kv_full[st], (kt / NST) & 1))) break;
+        const uint32_t ksl = (2 * kt) % NSL;
+        if (!(ok = wait1(&kv_full[ksl], ((2 * kt) / NSL) & 1))) break;
+        if (pact[0] || pact[1]) {  // the previous tile's V
+          if (!(ok = wait1(&kv_full[pvs], ((2 * kt - 1) / NSL) & 1))) break;
+        }
+        if (lane == 0) fence_proxy_async_smem();  // the slots were written by cp.async (generic proxy)
         const bool act[2] = {j < g.nt0, g.t1};
-        const uint32_t k_addr = smem_u32(smem + C::kStageOff + st * C::kStageB);
+        const uint32_t k_addr = smem_u32(smem + C::kStageOff + ksl * C::kKB);
 #pragma unroll
         for (int qi = 0; qi < 2; ++qi) {
-          if (!act[qi] || !ok) continue;
-          const uint32_t c = cnt[qi];
-          // the softmax warps hold the previous S of this Q tile in registers
-          if (c >= 1 && !(ok = wait1(&s_free[qi], (c - 1) & 1))) break;
-          if (lane == 0) {
-            tc::fence_after_sync();
+          if (pact[qi]) {
+            if (!(ok = issue_pv(qi, pvs, pc[qi], acc[qi]))) break;
+            acc[qi] = true;
+          }
+          if (act[qi] && lane == 0) {
             const uint32_t qa0 = q_addr + qi * C::kQTileB;
 #pragma unroll
             for (int kk = 0; kk < D / 16; ++kk) {
               const uint32_t off_q = (kk >> 2) * (128 * 128) + (kk & 3) * 32;
               const uint32_t off_k = (kk >> 2) * (kBN * 128) + (kk & 3) * 32;
-              tc::mma_bf16(tmem + qi * 64, tc::sw128_desc(qa0 + off_q, 16, 1024),
+              tc::mma_bf16(tmem + qi * 128, tc::sw128_desc(qa0 + off_q, 16, 1024),
                            tc::sw128_desc(k_addr + off_k, 16, 1024), C::kIdescS, kk > 0);
             }
             tc::commit(&s_full[qi]);
           }
         }
         if (!ok) break;
-        if (j == g.j_hi - 1 && lane == 0) tc::commit(q_empty);  // Q is free once these scores are done
-        // keys at or beyond L inside this tile: zero their stale V rows
-        const int kbase = j * kBN;
-        if (g.L - kbase < kBN) {
-          const int z0 = g.L - kbase;
-          const int z1 = min(kBN, (g.L + BS - 1) / BS * BS - kbase);
-          uint8_t* vs = smem + C::kStageOff + st * C::kStageB + C::kKB;
-          const int n16 = (z1 - z0) * 8;  // 16-byte chunks per half
-          for (int i = lane; i < n16 * C::kHalves; i += 32) {
-            const int h = i / n16, rem = i - h * n16;
-            *reinterpret_cast<uint4*>(vs + h * kBN * 128 + (z0 + rem / 8) * 128 + (rem & 7) * 16) =
-                make_uint4(0u, 0u, 0u, 0u);
-          }
-          fence_proxy_async_smem();
-          __syncwarp();
+        if (lane == 0) {
+          tc::commit(&kv_empty[ksl]);                             // K(j) is consumed once S(j) is done
+          if (pact[0] || pact[1]) tc::commit(&kv_empty[pvs]);     // V of the previous tile
+          if (j == g.j_hi - 1) tc::commit(q_empty);               // every product reading Q is issued
         }
-        if (have_prev && !(ok = issue_pv(pst, pact, pc, first))) break;
-        have_prev = true;
-        pst = st;
 #pragma unroll
         for (int qi = 0; qi < 2; ++qi) {
           pact[qi] = act[qi];
-          pc[qi] = cnt[qi];
-          cnt[qi] += act[qi] ? 1 : 0;
+          pc[qi] = ns[qi];
+          ns[qi] += act[qi] ? 1 : 0;
+        }
+        pvs = (2 * kt + 1) % NSL;
+      }
+      if (!ok) break;
+      // the last key tile's products
+      if (!(ok = wait1(&kv_full[pvs], ((2 * kt - 1) / NSL) & 1))) break;
+      if (lane == 0) fence_proxy_async_smem();
+#pragma unroll
+      for (int qi = 0; qi < 2; ++qi) {
+        if (pact[qi]) {
+          if (!(ok = issue_pv(qi, pvs, pc[qi], acc[qi]))) break;
         }
       }
-      if (ok && have_prev) ok = issue_pv(pst, pact, pc, first);
+      if (!ok) break;
+      if (lane == 0) tc::commit(&kv_empty[pvs]);
     }
     // no MMA may be in flight when TMEM is released
     if (lane == 0) {
@@ -406,24 +463,26 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     __syncwarp();
   } else {
+    setmaxnreg_inc<kRegSoftmax>();
     // ================= softmax: warps 4 qi .. 4 qi + 3 own Q tile qi, one row per thread
     const int qi = warp >> 2;
     const int r = tid & 127;
     const uint32_t t_lane = tmem + (static_cast<uint32_t>((warp & 3) * 32) << 16);
+    const uint32_t s_col = qi * 128;
     const uint32_t o_col = C::kOCol + qi * D;
-    uint32_t cnt = 0;
+    uint32_t cnt = 0;  // S tiles of this Q tile consumed so far
     bool failed = false;
     for (int64_t b = beg; b < end && !failed;) {
       PSeg g;
       locate<GH>(b, beg, end, cta, prefix, S, HGp, a, g);
-      b += g.j_hi - g.j_lo;
+      b += g.adv;
+      if (g.j_lo == g.j_hi) continue;  // only fixed-cost units of a pair
       const int tok = g.pt * C::kPairTok + qi * C::kTOK + r / GH;
       const int lim = min(g.L - g.ql + tok, g.L - 1);  // last key this row may see
       const int jend = qi == 0 ? min(g.j_hi, g.nt0) : (g.t1 ? g.j_hi : g.j_lo);
       float m_used = -CUDART_INF_F, l = 0.f;
       int done = 0;
       for (int j = g.j_lo; j < jend; ++j) {
-        const uint32_t bb = cnt & 1;
         failed = !mbar_wait(&s_full[qi], cnt & 1, a.status, a.wait_limit_ns);
         if (__any_sync(0xffffffffu, failed)) {
           failed = true;
@@ -431,13 +490,9 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         tc::fence_after_sync();
         float sv[kBN];
-        tc::ld32(t_lane + qi * 64, sv);
-        tc::ld32(t_lane + qi * 64 + 32, sv + 32);
+#pragma unroll
+        for (int q = 0; q < kBN / 32; ++q) tc::ld32(t_lane + s_col + 32 * q, sv + 32 * q);
         tc::wait_ld();
-        // S is in registers: the next scores of this Q tile may be computed now
-        tc::fence_before_sync();
-        __syncwarp();
-        if (lane == 0) mbar_arrive(&s_free[qi]);
         const int kbase = j * kBN;
         // With a positive scale the row max is taken on the raw scores and the
         // scale is folded into the exponent's FMA below; the causal mask is
@@ -471,15 +526,30 @@ __global__ void __launch_bounds__(kThreads, 1)
           alpha = fast_exp2(m_used - m_new);
           m_used = m_new;
         }
-        if (done > 0 && __any_sync(0xffffffffu, bump)) {
-          // O holds the P.V products up to the previous tile: wait, then rescale
-          const uint32_t pb = (cnt - 1) & 1;
-          failed = !mbar_wait(&pv_done[qi * 2 + pb], ((cnt - 1) >> 1) & 1, a.status, a.wait_limit_ns);
-          if (__any_sync(0xffffffffu, failed)) {
-            failed = true;
-            break;
+        l *= alpha;
+        // a row that sees no key of this segment yet keeps m = -inf: its
+        // probabilities are exactly 0 (exp2 of -inf)
+        const float m_e = m_used == -CUDART_INF_F ? 0.f : m_used;
+        // P over the first 64 columns of this tile's S (already in registers)
+        float2 lq = make_float2(0.f, 0.f);
+        const float2 sc2 = make_float2(sc, sc), nm2 = make_float2(-m_e, -m_e);
+#pragma unroll
+        for (int q = 0; q < kBN / 32; ++q) {
+          uint32_t pk[16];
+#pragma unroll
+          for (int i = 0; i < 16; ++i) {
+            const float2 x = __ffma2_rn(make_float2(sv[32 * q + 2 * i], sv[32 * q + 2 * i + 1]), sc2, nm2);
+            const float2 e = make_float2(ex2_ftz(x.x), ex2_ftz(x.y));
+            lq = __fadd2_rn(lq, e);
+            const __nv_bfloat162 h2 = __floats2bfloat162_rn(e.x, e.y);
+            pk[i] = *reinterpret_cast<const uint32_t*>(&h2);
           }
-          tc::fence_after_sync();
+          tc::st16u(t_lane + s_col + 16 * q, pk);
+        }
+        l += lq.x + lq.y;
+        // O holds every product up to the previous tile (a completed S implies
+        // the earlier P.V completed): rescale it before this tile's product
+        if (j > g.j_lo && __any_sync(0xffffffffu, bump)) {
 #pragma unroll 1
           for (int q = 0; q < D / 32; ++q) {
             float ov[32];
@@ -489,42 +559,18 @@ __global__ void __launch_bounds__(kThreads, 1)
             for (int i = 0; i < 32; ++i) ov[i] *= alpha;
             tc::st32(t_lane + o_col + 32 * q, ov);
           }
-          tc::wait_st();
         }
-        l *= alpha;
-        // a row that sees no key of this segment yet keeps m = -inf: its
-        // probabilities are exactly 0 (exp2 of -inf)
-        const float m_e = m_used == -CUDART_INF_F ? 0.f : m_used;
-        uint32_t pk[kBN / 2];
-        float lq[4] = {0.f, 0.f, 0.f, 0.f};
-#pragma unroll
-        for (int i = 0; i < kBN / 2; ++i) {
-          const float p0 = fast_exp2(fmaf(sv[2 * i], sc, -m_e));
-          const float p1 = fast_exp2(fmaf(sv[2 * i + 1], sc, -m_e));
-          lq[i & 3] += p0 + p1;
-          const __nv_bfloat162 h2 = __floats2bfloat162_rn(p0, p1);
-          pk[i] = *reinterpret_cast<const uint32_t*>(&h2);
-        }
-        l += (lq[0] + lq[1]) + (lq[2] + lq[3]);
-        if (cnt >= 2) {  // P buffer bb was last read by P.V product cnt - 2
-          failed = !mbar_wait(&pv_done[qi * 2 + bb], ((cnt - 2) >> 1) & 1, a.status, a.wait_limit_ns);
-          if (__any_sync(0xffffffffu, failed)) {
-            failed = true;
-            break;
-          }
-        }
-        tc::st32u(t_lane + C::kPCol + qi * 64 + bb * 32, pk);
         tc::wait_st();
         tc::fence_before_sync();
         __syncwarp();
-        if (lane == 0) mbar_arrive(&p_full[qi * 2 + bb]);
+        if (lane == 0) mbar_arrive(&p_full[qi]);
         ++cnt;
         ++done;
       }
       if (failed) break;
       if (done > 0) {
-        const uint32_t pb = (cnt - 1) & 1;
-        failed = !mbar_wait(&pv_done[qi * 2 + pb], ((cnt - 1) >> 1) & 1, a.status, a.wait_limit_ns);
+        // the segment's last product of this Q tile is number cnt - 1
+        failed = !mbar_wait(&pv_done[qi], (cnt - 1) & 1, a.status, a.wait_limit_ns);
         if (__any_sync(0xffffffffu, failed)) {
           failed = true;
           break;
@@ -605,9 +651,9 @@ __global__ void __launch_bounds__(256) prefill_combine_kernel(const PrefillArgs 
   const int64_t beg = static_cast<int64_t>(c) * T / Geff, end = static_cast<int64_t>(c + 1) * T / Geff;
   PSeg g;
   locate<GH>(end - 1, beg, end, c, prefix, S, a.num_q_heads / GH, a, g);
-  const int64_t ps = (end - 1) - g.j_lo;  // the pair's first and one-past-last global tile
+  const int64_t ps = g.tile0;  // the pair's first and one-past-last key-tile unit
   const int64_t pe = ps + g.nt;
-  if (pe <= end || ps < beg) return;      // not split after this CTA, or not started by it
+  if (end - 1 < ps || pe <= end || ps < beg) return;  // no tile here, not split after this CTA, or not started by it
   const int c1 = cta_of_block(pe - 1, T, Geff);
   const int row = blockIdx.y * 32 + (threadIdx.x >> 3);
   const int qi = row >> 7, rr = row & 127;
@@ -618,7 +664,7 @@ __global__ void __launch_bounds__(256) prefill_combine_kernel(const PrefillArgs 
 #pragma unroll
   for (int i = 0; i < kCols; ++i) acc[i] = 0.f;
   for (int cc = c; cc <= c1; ++cc) {
-    const int slot = cc == c ? 2 * c + (ps > beg ? 1 : 0) : 2 * cc;
+    const int slot = cc == c ? 2 * c + 1 : 2 * cc;
     const size_t sr = static_cast<size_t>(slot) * 256 + row;
     const float lse = a.pf_lse[sr];
     if (lse == -CUDART_INF_F) continue;
@@ -712,7 +758,7 @@ int32_t prefill_grid(int32_t num_seqs, int32_t num_q_heads, int32_t num_kv_heads
   const int64_t gh = prefill_heads_per_tile(num_q_heads / num_kv_heads);
   const int64_t pair_tok = 2 * (128 / gh);
   const int64_t pairs = static_cast<int64_t>(num_seqs) * (num_q_heads / gh) * ((max_query_len + pair_tok - 1) / pair_tok);
-  const int64_t tiles = pairs * ((static_cast<int64_t>(max_context_len) + kBN - 1) / kBN);
+  const int64_t tiles = pairs * (kSegUnits + (static_cast<int64_t>(max_context_len) + kBN - 1) / kBN);
   int64_t g = (tiles + kMinTilesPerCta - 1) / kMinTilesPerCta;
   if (g > num_sms()) g = num_sms();
   return static_cast<int32_t>(g < 1 ? 1 : g);
