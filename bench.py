@@ -546,21 +546,47 @@ def prefill_only_call(b):
 
 SWEEP = ("tiny", "gqa_long", "prefix_cow", "mixed_bs8", "mixed_bs16", "mixed_bs32")
 L2_FLUSH_BYTES = 512 << 20   # > 4x the 126 MB L2
+L2_BYTES = 126 << 20
+
+
+def rotated_copies(b, touched_bytes: int):
+    """Copies of a prepared batch with their own KV caches, queries and outputs
+    (same values), enough that the copies other than the one being called
+    hold at least 3x the L2 of the data a call reads, so the called copy's
+    data has been evicted since its last use: a cold L2 without the dirty
+    lines a flush by writing leaves behind. None when that needs more than 8."""
+    import dataclasses
+    r = -(-3 * L2_BYTES // max(int(touched_bytes), 1)) + 1
+    if r > 8:
+        return None
+    return [b] + [dataclasses.replace(b, k_cache=b.k_cache.clone(), v_cache=b.v_cache.clone(), q=b.q.clone(),
+                                      out=b.out.clone()) for _ in range(max(r, 2) - 1)]
 
 
 def timed_calls(fn, reps: int, flush=None):
     """Each of ``reps`` calls timed alone with CUDA events on the current
-    stream; before each one ``flush`` (a write of L2_FLUSH_BYTES) evicts the L2,
-    outside the timed interval. Returns median / p10 / p90 in ms."""
+    stream. ``fn`` is one call, or a list of calls on rotated copies of the
+    inputs taken in turn (so each call finds its data evicted from L2 by the
+    others). Before each call, outside the timed interval: with ``flush`` (two
+    buffers of L2_FLUSH_BYTES), a write of the first evicts the L2 and a read
+    of the second then evicts the first's dirty lines, so their write-back does
+    not land inside the call; without it, a short spin keeps the GPU busy while
+    the host enqueues the call, so the interval holds device time only.
+    Returns median / p10 / p90 in ms."""
     import torch
+    fns = fn if isinstance(fn, (list, tuple)) else [fn]
     ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(reps)]
-    fn()
+    for f in fns:
+        f()
     torch.cuda.synchronize()
     for i in range(reps):
         if flush is not None:
-            flush.fill_(i & 0x7F)
+            flush[0].fill_(i & 0x7F)
+            flush[2].copy_(flush[1].view(-1, 1 << 16).amax(dim=1))
+        else:
+            torch.cuda._sleep(200000)
         ev[i][0].record()
-        fn()
+        fns[i % len(fns)]()
         ev[i][1].record()
     torch.cuda.synchronize()
     t = sorted(a.elapsed_time(z) for a, z in ev)
@@ -579,13 +605,19 @@ def measure_config(name: str, hbm_peak: float, bf16_peak: float, flush, reps: in
     gs.run_step(b)
     torch.cuda.synchronize()
     work = step_work(wl, b.num_step_tokens, int(b.step_pairs.shape[0]))
-    t = timed_calls(lambda: gs.run_attention(b), reps, flush)
+    copies = rotated_copies(b, work["attn_bytes"])
+    if copies is not None:
+        t = timed_calls([(lambda c=c: gs.run_attention(c)) for c in copies], reps)
+        l2 = "rotated over %d copies of the KV caches, queries and outputs (the others hold >= 3x the L2); " \
+             "no flush" % len(copies)
+    else:
+        t = timed_calls(lambda: gs.run_attention(b), reps, flush)
+        l2 = "flushed before each call (%d MB write, then %d MB read)" % (L2_FLUSH_BYTES >> 20, L2_FLUSH_BYTES >> 20)
     ms = t["median_ms"]
     ent = {"attention_us": ms * 1e3, "p10_us": t["p10_ms"] * 1e3, "p90_us": t["p90_ms"] * 1e3, "reps": reps,
            "query_tokens_per_s": wl.num_q_tokens / (ms * 1e-3), "algorithmic_bytes": work["attn_bytes"],
            "gbs": work["attn_bytes"] / (ms * 1e-3) / 1e9,
-           "frac_of_hbm_peak": work["attn_bytes"] / (ms * 1e-3) / 1e9 / hbm_peak,
-           "l2": "flushed before each call (%d MB write)" % (L2_FLUSH_BYTES >> 20)}
+           "frac_of_hbm_peak": work["attn_bytes"] / (ms * 1e-3) / 1e9 / hbm_peak, "l2": l2}
     e = 2 if geo.dtype == "bf16" else 4
     tok_bytes = 2 * geo.num_kv_heads * geo.head_dim * e
     lens = b.host["context_lens"]
@@ -594,12 +626,16 @@ def measure_config(name: str, hbm_peak: float, bf16_peak: float, flush, reps: in
         fn, flops, npre, qt = po
         tp = timed_calls(fn, reps, flush)
         ent["prefill_only"] = {"seqs": npre, "q_tokens": qt, "flops": flops, "us": tp["median_ms"] * 1e3,
+                               "l2": "flushed before each call (%d MB write, then %d MB read)" % (L2_FLUSH_BYTES >> 20, L2_FLUSH_BYTES >> 20),
                                "tflops": flops / (tp["median_ms"] * 1e-3) / 1e12,
                                "frac_of_bf16_peak": flops / (tp["median_ms"] * 1e-3) / 1e12 / bf16_peak}
     plan = gs.plan_cascade(b) if all(q == 1 for q in wl.q_lens) else None
     if plan is not None and plan.num_groups:
         out = torch.empty_like(b.out)
-        tc_ = timed_calls(lambda: gs.run_attention_cascade(b, plan, out=out), reps, flush)
+        if copies is not None:
+            tc_ = timed_calls([(lambda c=c: gs.run_attention_cascade(c, plan, out=out)) for c in copies], reps)
+        else:
+            tc_ = timed_calls(lambda: gs.run_attention_cascade(b, plan, out=out), reps, flush)
         shared, groups = plan.host["shared"], plan.host["groups"]
         own = sum(int(L) - int(sh) * geo.block_size for L, sh in zip(lens, shared))
         once = sum(int(shared[f]) * geo.block_size for f, _ in groups)
@@ -613,7 +649,7 @@ def measure_config(name: str, hbm_peak: float, bf16_peak: float, flush, reps: in
         ent["frac_of_hbm_peak_unique"] = (unique + work["attn_bytes"] - work["attn_kv_bytes"]) / (ms * 1e-3) / 1e9 \
             / hbm_peak
     ent["device_flags"] = P.pa_read_device_flags(clear=True)
-    del b
+    del b, copies
     torch.cuda.empty_cache()
     if oracle:
         cpu, _ = time_oracle(wl, budget_s=0.0, min_steps=1, max_steps=1)
@@ -703,7 +739,9 @@ def main():
     configs = None
     if world == 1 and args.workload == "llama7b" and not args.no_sweep:
         import torch
-        flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=device)
+        flush = (torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=device),
+                 torch.ones(L2_FLUSH_BYTES, dtype=torch.uint8, device=device),
+                 torch.empty(L2_FLUSH_BYTES >> 16, dtype=torch.uint8, device=device))
         configs = {}
         with ClockSampler(gpu_index) as sweep_clocks:
             for name in SWEEP:

@@ -495,42 +495,51 @@ __global__ void __launch_bounds__(GH * D) decode_combine_kernel(const DecodeArgs
   const size_t slot0 = static_cast<size_t>(u) + c0;
   const size_t l1_row = (static_cast<size_t>(s) * a.num_q_heads + static_cast<size_t>(hg) * GH + gi) * a.l1_max_chunks;
   const int64_t Bt = static_cast<int64_t>(a.seq_prefix[a.num_seqs]) * HG;
-  // With more CTAs than blocks some CTAs in [c0, c0 + n2) stream nothing and
-  // wrote no partial: they get weight 0 (and their stale slot is never read).
-  auto streams = [&](int cc) {
-    return static_cast<int64_t>(cc) * Bt / a.grid < static_cast<int64_t>(cc + 1) * Bt / a.grid;
-  };
-  // Each thread folds its partials with a running max (weights 2^(lse - M));
-  // loads are issued four at a time, ahead of the arithmetic.
+  // Each thread folds its partials with a running max (weights 2^(lse - M)).
   float M = -CUDART_INF_F, sum = 0.f, acc = 0.f;
-  for (int j0 = 0; j0 < n; j0 += 4) {
-    float lse[4], val[4];
+  auto fold = [&](float lse, float val) {
+    if (lse == -CUDART_INF_F) return;
+    const float m_new = fmaxf(M, lse);
+    const float keep = fast_exp2(M - m_new), w = fast_exp2(lse - m_new);
+    sum = fmaf(sum, keep, w);
+    acc = fmaf(acc, keep, w * val);
+    M = m_new;
+  };
+  if (Bt >= a.grid) {
+    // every CTA in [c0, c0 + n2) streamed a block of the unit and wrote its
+    // partial; loads are issued four at a time, ahead of the arithmetic
+    for (int j0 = 0; j0 < n2; j0 += 4) {
+      float lse[4], val[4];
 #pragma unroll
-    for (int q = 0; q < 4; ++q) {
-      const int j = j0 + q;
-      lse[q] = -CUDART_INF_F;
-      val[q] = 0.f;
-      if (j < n2) {
-        if (streams(c0 + j)) {
+      for (int q = 0; q < 4; ++q) {
+        const int j = j0 + q;
+        lse[q] = -CUDART_INF_F;
+        val[q] = 0.f;
+        if (j < n2) {
           const size_t part = (slot0 + j) * GH + gi;
           lse[q] = a.part_lse[part];
           val[q] = a.part_o[part * D + d];
         }
-      } else if (j < n) {
-        lse[q] = a.l1_lse[l1_row + (j - n2)];
-        val[q] = a.l1_o[(l1_row + (j - n2)) * D + d];
       }
-    }
 #pragma unroll
-    for (int q = 0; q < 4; ++q) {
-      if (lse[q] == -CUDART_INF_F) continue;
-      const float m_new = fmaxf(M, lse[q]);
-      const float keep = fast_exp2(M - m_new), w = fast_exp2(lse[q] - m_new);
-      sum = fmaf(sum, keep, w);
-      acc = fmaf(acc, keep, w * val[q]);
-      M = m_new;
+      for (int q = 0; q < 4; ++q) fold(lse[q], val[q]);
+    }
+  } else if (n2 > 0) {
+    // more CTAs than blocks: some CTAs in [c0, c0 + n2) streamed nothing and
+    // wrote no partial (their stale slots are never read); the ones that did
+    // are the owners of the unit's blocks, in order
+    const int64_t ub0 = static_cast<int64_t>(a.seq_prefix[s]) * HG + static_cast<int64_t>(hg) * nbs;
+    int prev = -1;
+    for (int k = 0; k < nbs; ++k) {
+      const int c = cta_of_block(ub0 + k, Bt, a.grid);
+      if (c == prev) continue;
+      prev = c;
+      const size_t part = (slot0 + (c - c0)) * GH + gi;
+      fold(a.part_lse[part], a.part_o[part * D + d]);
     }
   }
+  for (int j = n2; j < n; ++j)  // prefix-pass partials of cascade decode
+    fold(a.l1_lse[l1_row + (j - n2)], a.l1_o[(l1_row + (j - n2)) * D + d]);
   const int row = __ldg(a.query_start_loc + s);
   static_cast<T*>(a.out)[(static_cast<size_t>(row) * a.num_q_heads + hg * GH + gi) * D + d] =
       Elem<T>::narrow(acc / sum);
@@ -561,6 +570,11 @@ cudaError_t launch_decode_t(DecodeArgs& a, const CUtensorMap& kmap, const CUtens
   const int per_sm = ctas_per_sm(reinterpret_cast<const void*>(kern), C::kThreads, smem, 8);
   int grid = num_sms() * per_sm;
   if (grid > decode_max_grid()) grid = decode_max_grid();
+  // no more CTAs than the blocks there can be to stream (a CTA without a block
+  // only costs its launch, and makes the merge skip over it)
+  const int64_t max_blocks = static_cast<int64_t>(a.num_seqs) * (a.num_q_heads / C::kHPU) *
+                             ((static_cast<int64_t>(a.max_context_len) + BS - 1) / BS);
+  if (grid > max_blocks) grid = static_cast<int>(max_blocks > 0 ? max_blocks : 1);
   if (const char* env = getenv("PA_DECODE_GRID")) {  // testing / tuning: cap the grid
     const int v = atoi(env);
     if (v >= 1 && v < grid) grid = v;
