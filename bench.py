@@ -45,9 +45,9 @@ UNIT = "query-tokens/s"
 # DRAM bytes (read + write) of one launch of the workload's decode kernel, from
 # `ncu --set full` captures (profiles/), valid while the kernel sources match.
 NCU_TRAFFIC = {
-    "sources": "6b946b56efe8fe52",   # decode kernel sources of the capture
-    "llama7b_decode_b32_bf16": 589813248 + 5480960,    # paged_decode_kernel
-    "gqa_long_decode_b16_bf16": 166979840 + 5190144,   # paged_decode_kernel
+    "sources": "6e723f454aaa9541",   # decode kernel sources of the capture
+    "llama7b_decode_b32_bf16": 589814528 + 4097536,    # paged_decode_kernel
+    "gqa_long_decode_b16_bf16": 167228416 + 6554880,   # paged_decode_kernel
 }
 
 

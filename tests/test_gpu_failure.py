@@ -30,10 +30,14 @@ def P():
     return P
 
 
-def test_bounded_wait_runs_out_and_reports(P):
+@pytest.mark.parametrize("name", ["gqa_long", "mixed_bs16"])
+def test_bounded_wait_runs_out_and_reports(P, name):
+    """gqa_long: decode rows only (the CUDA-core decode grid and the merge);
+    mixed_bs16: the prefill grid as well (its MMA, producer and softmax warps
+    all give up, then drain their own copies and MMAs before the CTA exits)."""
     import torch
     from paged_kv_cache_heads_b200 import scenario as gs
-    b = gs.prepare(W.gqa_long_decode())   # decode rows only: the CUDA-core decode grid and the merge
+    b = gs.prepare(W.CONFIGS[name]())
     gs.run_step(b)
     torch.cuda.synchronize()
     want = b.out.clone()

@@ -200,7 +200,7 @@ def _prefill_rows(qsl):
 
 def test_mixed_results_agree_across_block_sizes(P):
     """The block size must not change results ([A] §"块大小选择的工程权衡" treats
-    it as a tunable). Prefill rows are computed over 64-key tiles at every
+    it as a tunable). Prefill rows are computed over 128-key tiles at every
     block size, so the same tokens meet the same MMAs in the same tile
     positions and the rows must agree bit for bit; decode rows split their key
     ranges at block boundaries that do depend on the block size, so they agree
