@@ -345,7 +345,7 @@ bool workspace_layout(int32_t num_seqs, int32_t num_q_heads, int32_t max_query_l
     const size_t rows = size_t(2) * w->pf_grid * 256;
     w->pf_prefix_off = (w->bytes + 255) & ~size_t(255);
     w->pf_o_off = (w->pf_prefix_off + (size_t(num_seqs) + 3) * 4 + 255) & ~size_t(255);
-    w->pf_lse_off = (w->pf_o_off + rows * cache->head_dim * 4 + 255) & ~size_t(255);
+    w->pf_lse_off = (w->pf_o_off + rows * cache->head_dim * 2 + 255) & ~size_t(255);  // fp16 O / l rows
     w->bytes = w->pf_lse_off + rows * 4;
   }
   return true;
@@ -470,7 +470,7 @@ pa_status pa_attention(const void* q, const void* k_cache, const void* v_cache,
     p.l1_max_chunks = 0;
     p.l1_chunk_blocks = 1;
     p.pf_prefix = reinterpret_cast<int32_t*>(static_cast<char*>(workspace) + wl.pf_prefix_off);
-    p.pf_o = reinterpret_cast<float*>(static_cast<char*>(workspace) + wl.pf_o_off);
+    p.pf_o = reinterpret_cast<uint16_t*>(static_cast<char*>(workspace) + wl.pf_o_off);
     p.pf_lse = reinterpret_cast<float*>(static_cast<char*>(workspace) + wl.pf_lse_off);
     p.grid = wl.pf_grid;
     // K/V boxes are 64 columns wide (128 bytes) to match the 128-byte swizzle

@@ -74,9 +74,9 @@ struct PrefillArgs {
   // Prefill rows (workspace): key tiles before each sequence, then the grid
   // the tiles were split over and their total ([num_seqs + 3], written by the
   // kernel for the merge); partials of split work items, two slots per CTA of
-  // 256 rows each ([2 * grid][256][head_dim] and [2 * grid][256]).
+  // 256 rows each ([2 * grid][256][head_dim] fp16 and [2 * grid][256] fp32).
   int32_t* pf_prefix;
-  float* pf_o;
+  uint16_t* pf_o;               // partial O / l rows as IEEE fp16 bits
   float* pf_lse;
   int32_t grid;                // CTAs of the prefill grid (prefill_grid)
 };

@@ -42,6 +42,7 @@
 //    (TMEM lane = row), fp32 online softmax with exp2 on the scale folded into
 //    log2 e. O is rescaled in TMEM only when a row's running max grows by
 //    more than 2^8.
+#include <cuda_fp16.h>
 #include <math_constants.h>
 
 #include "decode_common.cuh"
@@ -615,11 +616,19 @@ __global__ void __launch_bounds__(kThreads, 1)
             tc::ld32(t_lane + o_col + 32 * q, ov);
             tc::wait_ld();
             if (row_ok && has) {
-              float* po = a.pf_o + srow * D + 32 * q;
+              // fp16 (11-bit significand, |O / l| <= max |V|): its rounding stays
+              // well under the bf16 rounding of the merged row
+              uint16_t* po = a.pf_o + srow * D + 32 * q;
 #pragma unroll
-              for (int v4 = 0; v4 < 8; ++v4)
-                *reinterpret_cast<float4*>(po + 4 * v4) = make_float4(
-                    ov[4 * v4] * inv_l, ov[4 * v4 + 1] * inv_l, ov[4 * v4 + 2] * inv_l, ov[4 * v4 + 3] * inv_l);
+              for (int v4 = 0; v4 < 4; ++v4) {
+                uint32_t pk[4];
+#pragma unroll
+                for (int i = 0; i < 4; ++i) {
+                  const __half2 h2 = __floats2half2_rn(ov[8 * v4 + 2 * i] * inv_l, ov[8 * v4 + 2 * i + 1] * inv_l);
+                  pk[i] = *reinterpret_cast<const uint32_t*>(&h2);
+                }
+                *reinterpret_cast<uint4*>(po + 8 * v4) = make_uint4(pk[0], pk[1], pk[2], pk[3]);
+              }
             }
           }
         }
@@ -670,12 +679,15 @@ __global__ void __launch_bounds__(256) prefill_combine_kernel(const PrefillArgs 
     if (lse == -CUDART_INF_F) continue;
     float v[kCols];
 #pragma unroll
-    for (int i = 0; i < kCols / 4; ++i) {
-      const float4 f = *reinterpret_cast<const float4*>(a.pf_o + sr * D + col0 + 4 * i);
-      v[4 * i] = f.x;
-      v[4 * i + 1] = f.y;
-      v[4 * i + 2] = f.z;
-      v[4 * i + 3] = f.w;
+    for (int i = 0; i < kCols / 8; ++i) {
+      const uint4 u = *reinterpret_cast<const uint4*>(a.pf_o + sr * D + col0 + 8 * i);
+      const uint32_t w4[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+      for (int k = 0; k < 4; ++k) {
+        const float2 f = __half22float2(*reinterpret_cast<const __half2*>(&w4[k]));
+        v[8 * i + 2 * k] = f.x;
+        v[8 * i + 2 * k + 1] = f.y;
+      }
     }
     const float m_new = fmaxf(M, lse);
     const float keep = fast_exp2(M - m_new), w = fast_exp2(lse - m_new);
