@@ -617,17 +617,19 @@ __global__ void __launch_bounds__(kThreads, 1)
             tc::wait_ld();
             if (row_ok && has) {
               // fp16 (11-bit significand, |O / l| <= max |V|): its rounding stays
-              // well under the bf16 rounding of the merged row
-              uint16_t* po = a.pf_o + srow * D + 32 * q;
+              // well under the bf16 rounding of the merged row. Layout
+              // [slot][column / 8][256 rows][8]: a warp's 32 rows of one 8-column
+              // group are 512 contiguous bytes, so each store is coalesced.
 #pragma unroll
               for (int v4 = 0; v4 < 4; ++v4) {
+                uint16_t* po = a.pf_o + ((static_cast<size_t>(g.slot) * (D / 8) + 4 * q + v4) * 256 + qi * 128 + r) * 8;
                 uint32_t pk[4];
 #pragma unroll
                 for (int i = 0; i < 4; ++i) {
                   const __half2 h2 = __floats2half2_rn(ov[8 * v4 + 2 * i] * inv_l, ov[8 * v4 + 2 * i + 1] * inv_l);
                   pk[i] = *reinterpret_cast<const uint32_t*>(&h2);
                 }
-                *reinterpret_cast<uint4*>(po + 8 * v4) = make_uint4(pk[0], pk[1], pk[2], pk[3]);
+                *reinterpret_cast<uint4*>(po) = make_uint4(pk[0], pk[1], pk[2], pk[3]);
               }
             }
           }
@@ -647,7 +649,9 @@ __global__ void __launch_bounds__(kThreads, 1)
 
 // Merge the partials of pairs split between CTAs: block x handles the pair
 // that CTA x starts and CTA x + 1 continues (if any); blockIdx.y selects 32 of
-// its 256 rows; 8 threads share a row. O = sum_k 2^(lse_k - M) O_k / sum_k 2^(lse_k - M).
+// its 256 rows; a warp's lanes are 32 consecutive rows of one group of D / 8
+// columns (so each partial load is 512 contiguous bytes).
+// O = sum_k 2^(lse_k - M) O_k / sum_k 2^(lse_k - M).
 template <int D, int GH>
 __global__ void __launch_bounds__(256) prefill_combine_kernel(const PrefillArgs a) {
   constexpr int TOK = 128 / GH, PT = 2 * TOK, kCols = D / 8;
@@ -664,11 +668,11 @@ __global__ void __launch_bounds__(256) prefill_combine_kernel(const PrefillArgs 
   const int64_t pe = ps + g.nt;
   if (end - 1 < ps || pe <= end || ps < beg) return;  // no tile here, not split after this CTA, or not started by it
   const int c1 = cta_of_block(pe - 1, T, Geff);
-  const int row = blockIdx.y * 32 + (threadIdx.x >> 3);
+  const int row = blockIdx.y * 32 + (threadIdx.x & 31);
   const int qi = row >> 7, rr = row & 127;
   const int tok = g.pt * PT + qi * TOK + rr / GH;
   if (tok >= g.ql) return;
-  const int col0 = (threadIdx.x & 7) * kCols;
+  const int col0 = (threadIdx.x >> 5) * kCols;
   float M = -CUDART_INF_F, sum = 0.f, acc[kCols];
 #pragma unroll
   for (int i = 0; i < kCols; ++i) acc[i] = 0.f;
@@ -680,7 +684,8 @@ __global__ void __launch_bounds__(256) prefill_combine_kernel(const PrefillArgs 
     float v[kCols];
 #pragma unroll
     for (int i = 0; i < kCols / 8; ++i) {
-      const uint4 u = *reinterpret_cast<const uint4*>(a.pf_o + sr * D + col0 + 8 * i);
+      const uint4 u = *reinterpret_cast<const uint4*>(
+          a.pf_o + ((static_cast<size_t>(slot) * (D / 8) + col0 / 8 + i) * 256 + row) * 8);
       const uint32_t w4[4] = {u.x, u.y, u.z, u.w};
 #pragma unroll
       for (int k = 0; k < 4; ++k) {
