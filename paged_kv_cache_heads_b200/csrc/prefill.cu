@@ -60,12 +60,13 @@ constexpr int kMinTilesPerCta = 8;  // a CTA gets at least this many key tiles o
 // segment (loading its Q tiles, the epilogue, refilling the pipeline), so that
 // a CTA whose range crosses many short pairs is given fewer key tiles.
 constexpr int kSegUnits = 2;
-// Warps 0-7 softmax, 8 MMA issue, 9-10 K producers, 11-12 V producers, 13-15
+// Warps 0-7 softmax, 8 MMA issue, 9-11 K producers, 12-14 V producers, 15
 // idle. Warpgroups 2-3 (warps 8-15) hand registers to warpgroups 0-1:
 // 8 * 32 * kRegSoftmax + 8 * 32 * kRegOther = 512 threads * 128 registers.
 constexpr int kThreads = 512;
 constexpr int kRegSoftmax = 184;
 constexpr int kRegOther = 72;
+constexpr int kGatherWarps = 3;  // producer warps per K (and per V) tile
 static_assert(8 * 32 * kRegSoftmax + 8 * 32 * kRegOther == kThreads * 128, "register split must match the launch");
 constexpr int kMmaWarp = 8;
 constexpr int kLoadWarp = 9;
@@ -83,7 +84,6 @@ struct PrefillCfg {
   static constexpr int kNSL = D == 128 ? 4 : 8;
   static constexpr int kBlk = kBN / BS;          // KV blocks per key tile
   static constexpr int kCPR = D / 8;             // 16-byte chunks per key row
-  static constexpr int kRPS = 64 / kCPR;  // rows a pair of producer warps copies per step
   static constexpr int kStageOff = 2 * kQTileB;
   static constexpr int kBarOff = kStageOff + kNSL * kKB;
   // q_full, q_empty, mma_done, kv_full[NSL], kv_empty[NSL], s_full[2], p_full[2], pv_done[2]
@@ -199,7 +199,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     mbar_init(q_empty, 1);
     mbar_init(mma_done, 1);
     for (int i = 0; i < NSL; ++i) {
-      mbar_init(&kv_full[i], 64);  // one arrival per lane of the producer pair that fills it
+      mbar_init(&kv_full[i], 32 * kGatherWarps);  // one arrival per lane of the warps that fill it
       mbar_init(&kv_empty[i], 1);
     }
     for (int i = 0; i < 2; ++i) {
@@ -268,25 +268,29 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   // Registers move from warpgroups 2-3 (MMA issue, producers, idle) to the
   // softmax warpgroups: each role calls setmaxnreg first thing.
-  if (warp >= kLoadWarp + 4) {
+  if (warp >= kLoadWarp + 2 * kGatherWarps) {
     setmaxnreg_dec<kRegOther>();  // idle warps only hand over their registers
   } else if (warp >= kLoadWarp) {
     setmaxnreg_dec<kRegOther>();
-    // ================= producers. Warps kLoadWarp, +1 gather every key tile's K,
-    // warps kLoadWarp + 2, +3 its V, each pair half of the rows (so each ring
-    // slot is filled by one pair, in order), with 16-byte cp.async copies into the 128-byte swizzled layout
-    // the MMAs read (chunk c of row r at r * 128 + ((c ^ (r & 7)) << 4) within
-    // its 64-column half); rows at or beyond L are filled with zeros, so stale
-    // bits in the unfilled tail of the last block never reach the MMAs. Every
-    // lane arrives on kv_full asynchronously, when its copies have landed; the
-    // MMA thread fences them for the tensor cores. The K warp also loads each
-    // segment's two Q tiles (TMA), after the segment's first K tile: the Q
-    // buffer frees only when the previous segment's last scores are done.
-    const int kv = (warp - kLoadWarp) >> 1;                 // 0: K, 1: V
-    const int p = ((warp - kLoadWarp) & 1) * 32 + lane;  // thread of the pair
-    const int ch = p % C::kCPR;  // 16-byte chunk of a row
-    const int rg = p / C::kCPR;  // first row of this thread; rows rg + kRPS i
-    const uint32_t dst_col = (ch >> 3) * (kBN * 128) + rg * 128;
+    // ================= producers. kGatherWarps warps gather every key tile's
+    // K, as many its V (so each ring slot is filled by the same warps, in
+    // order); warp w of a set takes the tile's rows in groups of 8 (w, w +
+    // kGatherWarps, ...), with 16-byte cp.async copies straight into the 128-byte swizzled
+    // layout the MMAs read (chunk c of row r at r * 128 + ((c ^ (r & 7)) << 4)
+    // within its 64-column half). Rows at or beyond L are filled with zeros, so
+    // stale bits in the unfilled tail of the last block never reach the MMAs.
+    // Every lane arrives on kv_full asynchronously, when its copies have
+    // landed; the MMA thread fences them for the tensor cores. The first K warp
+    // also loads each segment's two Q tiles (TMA), after the segment's first K
+    // tile: the Q buffer frees only when the previous segment's last scores are
+    // done. (More gathering warps keep more copies in flight: each warp
+    // sustains only a few bytes per cycle.)
+    const int kv = (warp - kLoadWarp) / kGatherWarps;     // 0: K, 1: V
+    const int wi = (warp - kLoadWarp) % kGatherWarps;     // warp within its set
+    constexpr int RPW = 32 / C::kCPR;                     // rows per warp step
+    const int ch = lane % C::kCPR;                        // 16-byte chunk of a row
+    const int rl = lane / C::kCPR;                        // row of the step
+    const uint32_t dst_col = (ch >> 3) * (kBN * 128);
     const int64_t tok_bytes = static_cast<int64_t>(a.num_kv_heads) * D * 2;
     bool ok = true;
     uint32_t kt = 0, nq = 0;  // key tiles and segments of this CTA so far
@@ -299,59 +303,54 @@ __global__ void __launch_bounds__(kThreads, 1)
       const int hq0 = g.hg * GH, hk = hq0 / G;
       const int* row = a.block_tables + static_cast<size_t>(g.s) * a.max_blocks_per_seq;
       const int nblk_valid = (g.L + BS - 1) / BS;
-      const char* kcol = static_cast<const char*>(a.k_cache) + static_cast<size_t>(hk) * D * 2 + ch * 16;
-      const char* vcol = static_cast<const char*>(a.v_cache) + static_cast<size_t>(hk) * D * 2 + ch * 16;
+      const char* src = static_cast<const char*>(kv ? a.v_cache : a.k_cache) + static_cast<size_t>(hk) * D * 2 +
+                        ch * 16;
       for (int j = g.j_lo; j < g.j_hi && ok; ++j, ++kt) {
-        // byte offset of this lane's first row (rg) in each block of the tile;
-        // -1: the block is past the sequence (or invalid) and its rows are zero-filled
-        int64_t boff[C::kBlk];
-#pragma unroll
-        for (int bb = 0; bb < C::kBlk; ++bb) {
-          const int lb = j * C::kBlk + bb;
-          boff[bb] = -1;
-          if (lb < nblk_valid) {
-            const int pb = __ldg(row + lb);
-            if (pb >= 0 && pb < a.num_blocks) boff[bb] = (static_cast<int64_t>(pb) * BS + rg) * tok_bytes;
-            else if (p == 0) raise_flag(a.status, PA_FLAG_BLOCK_RANGE);
-          }
-        }
         const int kbase = j * kBN;
-        const bool full = kbase + kBN <= g.L;  // every row of the tile is a live key
-        {
-          const uint32_t n = 2 * kt + kv, sl = n % NSL;
-          if (lane == 0) ok = mbar_wait(&kv_empty[sl], ((n / NSL) & 1) ^ 1, a.status, a.wait_limit_ns);
-          ok = __shfl_sync(0xffffffffu, ok, 0) != 0;
-          if (!ok) break;
-          const uint32_t dst = smem_u32(smem + C::kStageOff + sl * C::kKB) + dst_col;
-          const char* src = kv ? vcol : kcol;
+        const uint32_t n = 2 * kt + kv, sl = n % NSL;
+        if (lane == 0) ok = mbar_wait(&kv_empty[sl], ((n / NSL) & 1) ^ 1, a.status, a.wait_limit_ns);
+        ok = __shfl_sync(0xffffffffu, ok, 0) != 0;
+        if (!ok) break;
+        const uint32_t dst = smem_u32(smem + C::kStageOff + sl * C::kKB) + dst_col;
+        // the tile's 128 rows in groups of 8 (one block holds whole groups):
+        // warp wi takes groups wi, wi + kGatherWarps, ...
+        for (int rgp = wi; rgp < kBN / 8; rgp += kGatherWarps) {
+          const int lb = j * C::kBlk + (rgp * 8) / BS;
+          int pb = -1;  // -1: past the sequence (or invalid): the rows are zero-filled
+          if (lb < nblk_valid) {
+            pb = __ldg(row + lb);
+            if (pb < 0 || pb >= a.num_blocks) {
+              if (lane == 0 && kv == 1) raise_flag(a.status, PA_FLAG_BLOCK_RANGE);
+              pb = -1;
+            }
+          }
+          const char* bsrc = src + (pb >= 0 ? static_cast<int64_t>(pb) * BS * tok_bytes : 0);
 #pragma unroll
-          for (int i = 0; i < kBN / C::kRPS; ++i) {
-            const int r = rg + C::kRPS * i;
-            // rg < kRPS <= BS, so the block and the row's offset in it are known at compile time
-            const int64_t bo = boff[(C::kRPS * i) / BS];
-            const bool live = bo >= 0 && (full || kbase + r < g.L);
-            const int64_t off = bo + static_cast<int64_t>((C::kRPS * i) % BS) * tok_bytes;
-            cp_async16(dst + C::kRPS * i * 128 + (((ch & 7) ^ (r & 7)) << 4), src + (live ? off : 0),
+          for (int i = 0; i < 8 / RPW; ++i) {
+            const int r = rgp * 8 + rl + RPW * i;  // row of the tile
+            const int t = r % BS;                  // token of the block
+            const bool live = pb >= 0 && kbase + r < g.L;
+            cp_async16(dst + r * 128 + (((ch & 7) ^ (r & 7)) << 4), bsrc + (live ? t * tok_bytes : 0),
                        live ? 16u : 0u);
           }
-          cp_async_arrive(&kv_full[sl]);
-          if (warp == kLoadWarp && j == g.j_lo) {  // this segment's Q tiles
-            if (lane == 0) {
-              ok = mbar_wait(q_empty, (nq & 1) ^ 1, a.status, a.wait_limit_ns);
-              if (ok) {
-                mbar_arrive_expect_tx(q_full, 2 * C::kQTileB);
+        }
+        cp_async_arrive(&kv_full[sl]);
+        if (warp == kLoadWarp && j == g.j_lo) {  // this segment's Q tiles
+          if (lane == 0) {
+            ok = mbar_wait(q_empty, (nq & 1) ^ 1, a.status, a.wait_limit_ns);
+            if (ok) {
+              mbar_arrive_expect_tx(q_full, 2 * C::kQTileB);
 #pragma unroll
-                for (int qi = 0; qi < 2; ++qi)
+              for (int qi = 0; qi < 2; ++qi)
 #pragma unroll
-                  for (int h = 0; h < C::kHalves; ++h)
-                    tma_load_3d(smem + qi * C::kQTileB + h * 128 * 128, &qmap, q_full, h * 64, hq0,
-                                g.r0 + g.pt * C::kPairTok + qi * C::kTOK);
-              }
+                for (int h = 0; h < C::kHalves; ++h)
+                  tma_load_3d(smem + qi * C::kQTileB + h * 128 * 128, &qmap, q_full, h * 64, hq0,
+                              g.r0 + g.pt * C::kPairTok + qi * C::kTOK);
             }
-            ok = __shfl_sync(0xffffffffu, ok, 0) != 0;
-            if (!ok) break;
-            my_q = nq + 1;
           }
+          ok = __shfl_sync(0xffffffffu, ok, 0) != 0;
+          if (!ok) break;
+          my_q = nq + 1;
         }
       }
       ++nq;
