@@ -60,13 +60,13 @@ constexpr int kMinTilesPerCta = 8;  // a CTA gets at least this many key tiles o
 // segment (loading its Q tiles, the epilogue, refilling the pipeline), so that
 // a CTA whose range crosses many short pairs is given fewer key tiles.
 constexpr int kSegUnits = 2;
-// Warps 0-7 softmax, 8 MMA issue, 9-11 K producers, 12-14 V producers, 15
-// idle. Warpgroups 2-3 (warps 8-15) hand registers to warpgroups 0-1:
+// Warps 0-7 softmax, 8 MMA issue, 9-12 K producers, 13-15 V producers. Warpgroups 2-3 (warps 8-15) hand registers to warpgroups 0-1:
 // 8 * 32 * kRegSoftmax + 8 * 32 * kRegOther = 512 threads * 128 registers.
 constexpr int kThreads = 512;
 constexpr int kRegSoftmax = 184;
 constexpr int kRegOther = 72;
-constexpr int kGatherWarps = 3;  // producer warps per K (and per V) tile
+constexpr int kKWarps = 4;  // producer warps gathering each K tile
+constexpr int kVWarps = 3;  // and each V tile
 static_assert(8 * 32 * kRegSoftmax + 8 * 32 * kRegOther == kThreads * 128, "register split must match the launch");
 constexpr int kMmaWarp = 8;
 constexpr int kLoadWarp = 9;
@@ -199,7 +199,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     mbar_init(q_empty, 1);
     mbar_init(mma_done, 1);
     for (int i = 0; i < NSL; ++i) {
-      mbar_init(&kv_full[i], 32 * kGatherWarps);  // one arrival per lane of the warps that fill it
+      mbar_init(&kv_full[i], 32 * ((i & 1) ? kVWarps : kKWarps));  // one arrival per lane of the warps that fill it
       mbar_init(&kv_empty[i], 1);
     }
     for (int i = 0; i < 2; ++i) {
@@ -268,14 +268,14 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   // Registers move from warpgroups 2-3 (MMA issue, producers, idle) to the
   // softmax warpgroups: each role calls setmaxnreg first thing.
-  if (warp >= kLoadWarp + 2 * kGatherWarps) {
+  if (warp >= kLoadWarp + kKWarps + kVWarps) {
     setmaxnreg_dec<kRegOther>();  // idle warps only hand over their registers
   } else if (warp >= kLoadWarp) {
     setmaxnreg_dec<kRegOther>();
-    // ================= producers. kGatherWarps warps gather every key tile's
-    // K, as many its V (so each ring slot is filled by the same warps, in
-    // order); warp w of a set takes the tile's rows in groups of 8 (w, w +
-    // kGatherWarps, ...), with 16-byte cp.async copies straight into the 128-byte swizzled
+    // ================= producers. kKWarps warps gather every key tile's K and
+    // kVWarps its V (so each ring slot is filled by the same warps, in order);
+    // warp w of a set takes the tile's rows in groups of 8 (w, w + the set's
+    // size, ...), with 16-byte cp.async copies straight into the 128-byte swizzled
     // layout the MMAs read (chunk c of row r at r * 128 + ((c ^ (r & 7)) << 4)
     // within its 64-column half). Rows at or beyond L are filled with zeros, so
     // stale bits in the unfilled tail of the last block never reach the MMAs.
@@ -285,8 +285,9 @@ __global__ void __launch_bounds__(kThreads, 1)
     // tile: the Q buffer frees only when the previous segment's last scores are
     // done. (More gathering warps keep more copies in flight: each warp
     // sustains only a few bytes per cycle.)
-    const int kv = (warp - kLoadWarp) / kGatherWarps;     // 0: K, 1: V
-    const int wi = (warp - kLoadWarp) % kGatherWarps;     // warp within its set
+    const int kv = warp - kLoadWarp < kKWarps ? 0 : 1;          // 0: K, 1: V
+    const int wi = kv ? warp - kLoadWarp - kKWarps : warp - kLoadWarp;  // warp within its set
+    const int nw = kv ? kVWarps : kKWarps;
     constexpr int RPW = 32 / C::kCPR;                     // rows per warp step
     const int ch = lane % C::kCPR;                        // 16-byte chunk of a row
     const int rl = lane / C::kCPR;                        // row of the step
@@ -313,8 +314,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (!ok) break;
         const uint32_t dst = smem_u32(smem + C::kStageOff + sl * C::kKB) + dst_col;
         // the tile's 128 rows in groups of 8 (one block holds whole groups):
-        // warp wi takes groups wi, wi + kGatherWarps, ...
-        for (int rgp = wi; rgp < kBN / 8; rgp += kGatherWarps) {
+        // warp wi takes groups wi, wi + nw, ...
+        for (int rgp = wi; rgp < kBN / 8; rgp += nw) {
           const int lb = j * C::kBlk + (rgp * 8) / BS;
           int pb = -1;  // -1: past the sequence (or invalid): the rows are zero-filled
           if (lb < nblk_valid) {
