@@ -317,7 +317,7 @@ pa_status launch_decode_path(DecodeArgs& a, const void* q, const void* k_cache, 
 struct WorkspaceLayout {
   size_t bytes = 0, lse_off = 0, prefix_off = 0;
   // prefill rows: partition, partial outputs and their log-sum-exp
-  size_t pf_prefix_off = 0, pf_o_off = 0, pf_lse_off = 0;
+  size_t pf_split_off = 0, pf_o_off = 0, pf_lse_off = 0;
   int32_t pf_grid = 0;
 };
 bool workspace_layout(int32_t num_seqs, int32_t num_q_heads, int32_t max_query_len, int32_t max_context_len,
@@ -343,8 +343,8 @@ bool workspace_layout(int32_t num_seqs, int32_t num_q_heads, int32_t max_query_l
     // two partial slots of 256 rows per prefill CTA
     w->pf_grid = prefill_grid(num_seqs, num_q_heads, cache->num_kv_heads, max_query_len, max_context_len);
     const size_t rows = size_t(2) * w->pf_grid * 256;
-    w->pf_prefix_off = (w->bytes + 255) & ~size_t(255);
-    w->pf_o_off = (w->pf_prefix_off + (size_t(num_seqs) + 3) * 4 + 255) & ~size_t(255);
+    w->pf_split_off = (w->bytes + 255) & ~size_t(255);
+    w->pf_o_off = (w->pf_split_off + size_t(w->pf_grid) * 16 + 255) & ~size_t(255);
     w->pf_lse_off = (w->pf_o_off + rows * cache->head_dim * 2 + 255) & ~size_t(255);  // fp16 O / l rows
     w->bytes = w->pf_lse_off + rows * 4;
   }
@@ -469,7 +469,7 @@ pa_status pa_attention(const void* q, const void* k_cache, const void* v_cache,
     p.l1_lse = nullptr;
     p.l1_max_chunks = 0;
     p.l1_chunk_blocks = 1;
-    p.pf_prefix = reinterpret_cast<int32_t*>(static_cast<char*>(workspace) + wl.pf_prefix_off);
+    p.pf_split = reinterpret_cast<int4*>(static_cast<char*>(workspace) + wl.pf_split_off);
     p.pf_o = reinterpret_cast<uint16_t*>(static_cast<char*>(workspace) + wl.pf_o_off);
     p.pf_lse = reinterpret_cast<float*>(static_cast<char*>(workspace) + wl.pf_lse_off);
     p.grid = wl.pf_grid;
@@ -630,7 +630,7 @@ pa_status pa_attention_cascade(const void* q, const void* k_cache, const void* v
     p.l1_lse = reinterpret_cast<float*>(ws + wl.l1_lse_off);
     p.l1_max_chunks = max_chunks;
     p.l1_chunk_blocks = chunk_blocks;
-    p.pf_prefix = nullptr;
+    p.pf_split = nullptr;
     p.pf_o = nullptr;
     p.pf_lse = nullptr;
     p.grid = 0;

@@ -71,11 +71,12 @@ struct PrefillArgs {
   float* l1_lse;
   int32_t l1_max_chunks;
   int32_t l1_chunk_blocks;
-  // Prefill rows (workspace): key tiles before each sequence, then the grid
-  // the tiles were split over and their total ([num_seqs + 3], written by the
-  // kernel for the merge); partials of split work items, two slots per CTA of
-  // 256 rows each ([2 * grid][256][head_dim] fp16 and [2 * grid][256] fp32).
-  int32_t* pf_prefix;
+  // Prefill rows (workspace): per CTA, the work item it starts and the next
+  // CTAs continue ([grid]: first query row, rows left in the sequence, first
+  // query head, last covering CTA or -1), written by the kernel for the merge;
+  // partials of split work items, two slots per CTA of 256 rows each
+  // ([2 * grid][256][head_dim] fp16 and [2 * grid][256] fp32).
+  int4* pf_split;
   uint16_t* pf_o;               // partial O / l rows as IEEE fp16 bits
   float* pf_lse;
   int32_t grid;                // CTAs of the prefill grid (prefill_grid)

@@ -210,6 +210,11 @@ __global__ void __launch_bounds__(kThreads, 1)
     fence_barrier_init();
   }
   if (warp >= kLoadWarp && lane == 0) tma_prefetch_desc(&qmap);
+  // The merge grid chained after this one may be scheduled now: its CTAs take
+  // SMs as this grid's CTAs exit and wait there for this whole grid to finish,
+  // so the merge starts without a launch gap. (Every CTA of this grid is
+  // resident before any CTA can pass this point in all of them.)
+  launch_dependents();
 
   // ---- key tiles of every prefill sequence, and their prefix. This grid is
   // chained after the decode merge; every input it reads was complete before
@@ -243,12 +248,20 @@ __global__ void __launch_bounds__(kThreads, 1)
   __syncthreads();
   const int T = prefix[S];
   const int Geff = T > 0 ? min(static_cast<int>(gridDim.x), (T + kMinTilesPerCta - 1) / kMinTilesPerCta) : 1;
-  if (blockIdx.x == 0) {  // the partition, for the merge kernel
-    for (int i = tid; i <= S; i += blockDim.x) a.pf_prefix[i] = prefix[i];
-    if (tid == 0) {
-      a.pf_prefix[S + 1] = Geff;
-      a.pf_prefix[S + 2] = T;
+  // The work item this CTA starts and later CTAs continue, if any: the merge
+  // kernel's block for this CTA folds that item's partials together.
+  if (tid == 0) {
+    int4 rec = make_int4(0, 0, 0, -1);
+    if (T > 0 && static_cast<int>(blockIdx.x) < Geff) {
+      const int64_t b0 = static_cast<int64_t>(blockIdx.x) * T / Geff;
+      const int64_t e0 = static_cast<int64_t>(blockIdx.x + 1) * T / Geff;
+      PSeg g;
+      locate<GH>(e0 - 1, b0, e0, static_cast<int>(blockIdx.x), prefix, S, HGp, a, g);
+      const int64_t ps = g.tile0, pe = g.tile0 + g.nt;  // the item's first and one-past-last key-tile unit
+      if (e0 - 1 >= ps && pe > e0 && ps >= b0)
+        rec = make_int4(g.r0 + g.pt * C::kPairTok, g.ql - g.pt * C::kPairTok, g.hg * GH, cta_of_block(pe - 1, T, Geff));
     }
+    a.pf_split[blockIdx.x] = rec;
   }
   if (T == 0 || static_cast<int>(blockIdx.x) >= Geff) {
     if (tid == 0) grid_dependency_wait();  // finish no earlier than the previous grid
@@ -648,40 +661,37 @@ __global__ void __launch_bounds__(kThreads, 1)
 }
 
 // Merge the partials of pairs split between CTAs: block x handles the pair
-// that CTA x starts and CTA x + 1 continues (if any); blockIdx.y selects 32 of
-// its 256 rows; a warp's lanes are 32 consecutive rows of one group of D / 8
-// columns (so each partial load is 512 contiguous bytes).
+// that CTA x starts and CTAs x + 1 .. continue (its split record); blockIdx.y
+// selects 32 of its 256 rows; a warp's lanes are 32 consecutive rows of one
+// group of D / 8 columns (so each partial load is 512 contiguous bytes).
 // O = sum_k 2^(lse_k - M) O_k / sum_k 2^(lse_k - M).
 template <int D, int GH>
 __global__ void __launch_bounds__(256) prefill_combine_kernel(const PrefillArgs a) {
-  constexpr int TOK = 128 / GH, PT = 2 * TOK, kCols = D / 8;
-  grid_dependency_wait();  // the prefill grid (partials and the partition) is complete
-  const int S = a.num_seqs;
-  const int* prefix = a.pf_prefix;
-  const int Geff = prefix[S + 1], T = prefix[S + 2];
+  constexpr int TOK = 128 / GH, kCols = D / 8;
+  grid_dependency_wait();  // the prefill grid (partials and split records) is complete
   const int c = blockIdx.x;
-  if (c + 1 >= Geff) return;
-  const int64_t beg = static_cast<int64_t>(c) * T / Geff, end = static_cast<int64_t>(c + 1) * T / Geff;
-  PSeg g;
-  locate<GH>(end - 1, beg, end, c, prefix, S, a.num_q_heads / GH, a, g);
-  const int64_t ps = g.tile0;  // the pair's first and one-past-last key-tile unit
-  const int64_t pe = ps + g.nt;
-  if (end - 1 < ps || pe <= end || ps < beg) return;  // no tile here, not split after this CTA, or not started by it
-  const int c1 = cta_of_block(pe - 1, T, Geff);
+  const int4 rec = a.pf_split[c];  // first query row of the pair, rows left, first head, last CTA
+  if (rec.w < 0) return;
   const int row = blockIdx.y * 32 + (threadIdx.x & 31);
   const int qi = row >> 7, rr = row & 127;
-  const int tok = g.pt * PT + qi * TOK + rr / GH;
-  if (tok >= g.ql) return;
+  const int tok = qi * TOK + rr / GH;
+  if (tok >= rec.y) return;
   const int col0 = (threadIdx.x >> 5) * kCols;
-  float M = -CUDART_INF_F, sum = 0.f, acc[kCols];
+  // the pieces' log-sum-exps first (independent loads), then their rows
+  float M = -CUDART_INF_F;
+  for (int cc = c; cc <= rec.w; ++cc) {
+    const int slot = cc == c ? 2 * c + 1 : 2 * cc;
+    M = fmaxf(M, a.pf_lse[static_cast<size_t>(slot) * 256 + row]);
+  }
+  float sum = 0.f, acc[kCols];
 #pragma unroll
   for (int i = 0; i < kCols; ++i) acc[i] = 0.f;
-  for (int cc = c; cc <= c1; ++cc) {
+  for (int cc = c; cc <= rec.w; ++cc) {
     const int slot = cc == c ? 2 * c + 1 : 2 * cc;
-    const size_t sr = static_cast<size_t>(slot) * 256 + row;
-    const float lse = a.pf_lse[sr];
-    if (lse == -CUDART_INF_F) continue;
-    float v[kCols];
+    const float lse = a.pf_lse[static_cast<size_t>(slot) * 256 + row];
+    if (lse == -CUDART_INF_F) continue;  // no key of this piece reaches the row: its O was not written
+    const float w = fast_exp2(lse - M);
+    sum += w;
 #pragma unroll
     for (int i = 0; i < kCols / 8; ++i) {
       const uint4 u = *reinterpret_cast<const uint4*>(
@@ -690,20 +700,14 @@ __global__ void __launch_bounds__(256) prefill_combine_kernel(const PrefillArgs 
 #pragma unroll
       for (int k = 0; k < 4; ++k) {
         const float2 f = __half22float2(*reinterpret_cast<const __half2*>(&w4[k]));
-        v[8 * i + 2 * k] = f.x;
-        v[8 * i + 2 * k + 1] = f.y;
+        acc[8 * i + 2 * k] = fmaf(w, f.x, acc[8 * i + 2 * k]);
+        acc[8 * i + 2 * k + 1] = fmaf(w, f.y, acc[8 * i + 2 * k + 1]);
       }
     }
-    const float m_new = fmaxf(M, lse);
-    const float keep = fast_exp2(M - m_new), w = fast_exp2(lse - m_new);
-    sum = fmaf(sum, keep, w);
-#pragma unroll
-    for (int i = 0; i < kCols; ++i) acc[i] = fmaf(acc[i], keep, w * v[i]);
-    M = m_new;
   }
   const float inv = 1.f / sum;
   __nv_bfloat16* orow = static_cast<__nv_bfloat16*>(a.out) +
-                        (static_cast<size_t>(g.r0 + tok) * a.num_q_heads + g.hg * GH + rr % GH) * D + col0;
+                        (static_cast<size_t>(rec.x + tok) * a.num_q_heads + rec.z + rr % GH) * D + col0;
 #pragma unroll
   for (int i = 0; i < kCols / 8; ++i) {
     uint32_t pk[4];
