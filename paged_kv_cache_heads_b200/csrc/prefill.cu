@@ -677,32 +677,55 @@ __global__ void __launch_bounds__(256) prefill_combine_kernel(const PrefillArgs 
   const int tok = qi * TOK + rr / GH;
   if (tok >= rec.y) return;
   const int col0 = (threadIdx.x >> 5) * kCols;
-  // the pieces' log-sum-exps first (independent loads), then their rows
-  float M = -CUDART_INF_F;
-  for (int cc = c; cc <= rec.w; ++cc) {
-    const int slot = cc == c ? 2 * c + 1 : 2 * cc;
-    M = fmaxf(M, a.pf_lse[static_cast<size_t>(slot) * 256 + row]);
-  }
-  float sum = 0.f, acc[kCols];
+  const int np = rec.w - c + 1;  // pieces: this CTA's (slot 2c + 1), then slot 2cc of CTA cc
+  auto slot_of = [&](int k) { return k == 0 ? 2 * c + 1 : 2 * (c + k); };
+  float M = -CUDART_INF_F, sum = 0.f, acc[kCols];
 #pragma unroll
   for (int i = 0; i < kCols; ++i) acc[i] = 0.f;
-  for (int cc = c; cc <= rec.w; ++cc) {
-    const int slot = cc == c ? 2 * c + 1 : 2 * cc;
-    const float lse = a.pf_lse[static_cast<size_t>(slot) * 256 + row];
-    if (lse == -CUDART_INF_F) continue;  // no key of this piece reaches the row: its O was not written
+  // O += w f, skipping a piece no key of which reaches the row (its O was not written)
+  auto fold = [&](float lse, const uint4* u) {
+    if (lse == -CUDART_INF_F) return;
     const float w = fast_exp2(lse - M);
     sum += w;
 #pragma unroll
     for (int i = 0; i < kCols / 8; ++i) {
-      const uint4 u = *reinterpret_cast<const uint4*>(
-          a.pf_o + ((static_cast<size_t>(slot) * (D / 8) + col0 / 8 + i) * 256 + row) * 8);
-      const uint32_t w4[4] = {u.x, u.y, u.z, u.w};
+      const uint32_t w4[4] = {u[i].x, u[i].y, u[i].z, u[i].w};
 #pragma unroll
       for (int k = 0; k < 4; ++k) {
         const float2 f = __half22float2(*reinterpret_cast<const __half2*>(&w4[k]));
         acc[8 * i + 2 * k] = fmaf(w, f.x, acc[8 * i + 2 * k]);
         acc[8 * i + 2 * k + 1] = fmaf(w, f.y, acc[8 * i + 2 * k + 1]);
       }
+    }
+  };
+  auto load_row = [&](int slot, uint4* u) {
+#pragma unroll
+    for (int i = 0; i < kCols / 8; ++i)
+      u[i] = *reinterpret_cast<const uint4*>(a.pf_o + ((static_cast<size_t>(slot) * (D / 8) + col0 / 8 + i) * 256 + row) * 8);
+  };
+  constexpr int kMaxP = 4;
+  if (np <= kMaxP) {
+    // every load of the thread issued at once (a row not written is loaded but never used)
+    float lse[kMaxP];
+    uint4 u[kMaxP][kCols / 8];
+#pragma unroll
+    for (int k = 0; k < kMaxP; ++k) {
+      lse[k] = -CUDART_INF_F;
+      if (k < np) {
+        lse[k] = a.pf_lse[static_cast<size_t>(slot_of(k)) * 256 + row];
+        load_row(slot_of(k), u[k]);
+      }
+    }
+#pragma unroll
+    for (int k = 0; k < kMaxP; ++k) M = fmaxf(M, lse[k]);
+#pragma unroll
+    for (int k = 0; k < kMaxP; ++k) fold(lse[k], u[k]);
+  } else {
+    for (int k = 0; k < np; ++k) M = fmaxf(M, a.pf_lse[static_cast<size_t>(slot_of(k)) * 256 + row]);
+    for (int k = 0; k < np; ++k) {
+      uint4 u[kCols / 8];
+      load_row(slot_of(k), u);
+      fold(a.pf_lse[static_cast<size_t>(slot_of(k)) * 256 + row], u);
     }
   }
   const float inv = 1.f / sum;
