@@ -45,9 +45,9 @@ UNIT = "query-tokens/s"
 # DRAM bytes (read + write) of one launch of the workload's decode kernel, from
 # `ncu --set full` captures (profiles/), valid while the kernel sources match.
 NCU_TRAFFIC = {
-    "sources": "7c4b21b4fe262b29",   # decode kernel sources of the capture
-    "llama7b_decode_b32_bf16": 589814528 + 4418304,    # paged_decode_kernel
-    "gqa_long_decode_b16_bf16": 167221248 + 7170560,   # paged_decode_kernel
+    "sources": "14c46f4317e3d7af",   # decode kernel sources of the capture
+    "llama7b_decode_b32_bf16": 589856000 + 4239616,    # paged_decode_kernel
+    "gqa_long_decode_b16_bf16": 167207680 + 5744640,   # paged_decode_kernel
 }
 
 
