@@ -265,6 +265,17 @@ def test_prefill_only_batch_and_full_prompt(P):
     _check_attention(got, o.out, W.BF16, "prefill only")
 
 
+@pytest.mark.parametrize("q_len,ctx", [(64, 6000), (200, 2500)])
+def test_prefill_long_context_split_over_many_ctas(P, q_len, ctx):
+    """One prefill chunk on a long context, so few work items of many key
+    tiles: (64, 6000) spreads each item over about seven CTAs (the merge's
+    general path, more than four pieces), (200, 2500) over three or four."""
+    wl = W.random_case(5150 + q_len, num_seqs=2, q_lens=[q_len, 1], ctx_extra=[ctx, 300], num_kv_heads=2,
+                       group=4, head_dim=128, block_size=16, dtype=W.BF16)
+    b, o, got = _run_both(P, wl)
+    _check_attention(got, o.out, W.BF16, "long-context prefill q_len=%d ctx=%d" % (q_len, ctx))
+
+
 def test_prefill_large_logits_trigger_rescale(P):
     """Keys scaled so the running max grows tile after tile (exercises the O rescale)."""
     wl = W.random_case(41, num_seqs=2, q_lens=[96, 40], ctx_extra=[700, 300], num_kv_heads=2, group=4,
