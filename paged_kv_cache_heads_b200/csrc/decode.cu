@@ -157,11 +157,14 @@ __global__ void __launch_bounds__((NCW + 1) * 32, (GH == 1 ? 4 : PA_DECODE_GQA_C
       const int ql = __ldg(a.query_start_loc + s + 1) - r0;
       clen[s] = L;
       qrow[s] = r0;
-      const int skip = (ql == 1 && a.skip_blocks) ? __ldg(a.skip_blocks + s) : 0;
-      n = decode_blocks<BS>(L, ql, skip, a);
-      if (n < 0) {
-        raise_flag(a.status, PA_FLAG_CONTEXT_RANGE);
-        n = 0;
+      if (ql == 1) {
+        const int skip = a.skip_blocks ? __ldg(a.skip_blocks + s) : 0;
+        if (L < 1 || L > a.max_context_len || L > a.max_blocks_per_seq * BS || skip < 0 ||
+            skip > (L + BS - 1) / BS) {
+          raise_flag(a.status, PA_FLAG_CONTEXT_RANGE);
+        } else {
+          n = (L + BS - 1) / BS - skip;
+        }
       }
     }
     int total;
@@ -470,21 +473,14 @@ __global__ void __launch_bounds__((NCW + 1) * 32, (GH == 1 ? 4 : PA_DECODE_GQA_C
 template <typename T, int D, int BS, int GH>  // GH here: query heads per unit
 __global__ void __launch_bounds__(GH * D) decode_combine_kernel(const DecodeArgs a) {
   launch_dependents();
+  grid_dependency_wait();  // the decode grid (partials and the block prefix) is complete
   const int HG = a.num_q_heads / GH;
   const int u = blockIdx.x;
   const int s = u / HG, hg = u - s * HG;
-  // Before the wait, from the call's inputs (complete before the decode grid
-  // passed its own wait, which came before this grid could start): the
-  // sequence's decode blocks by the decode grid's rule, its shared blocks and
-  // its output row.
-  const int L = __ldg(a.context_lens + s);
-  const int row = __ldg(a.query_start_loc + s);
-  const int ql = __ldg(a.query_start_loc + s + 1) - row;
+  const int nbs = a.seq_prefix[s + 1] - a.seq_prefix[s];
   const int skip = a.skip_blocks ? __ldg(a.skip_blocks + s) : 0;
-  const int nbs = max(decode_blocks<BS>(L, ql, skip, a), 0);
   const int n1 = skip > 0 ? (skip + a.l1_chunk_blocks - 1) / a.l1_chunk_blocks : 0;  // prefix-pass chunks
   if (nbs == 0 && n1 == 0) return;
-  grid_dependency_wait();  // the decode grid (partials and the block prefix) is complete
   int c0 = 0, n2 = 0;  // covering decode CTAs c0 .. c0 + n2 - 1
   if (nbs > 0) {
     const int64_t B = static_cast<int64_t>(a.seq_prefix[a.num_seqs]) * HG;
@@ -544,6 +540,7 @@ __global__ void __launch_bounds__(GH * D) decode_combine_kernel(const DecodeArgs
   }
   for (int j = n2; j < n; ++j)  // prefix-pass partials of cascade decode
     fold(a.l1_lse[l1_row + (j - n2)], a.l1_o[(l1_row + (j - n2)) * D + d]);
+  const int row = __ldg(a.query_start_loc + s);
   static_cast<T*>(a.out)[(static_cast<size_t>(row) * a.num_q_heads + hg * GH + gi) * D + d] =
       Elem<T>::narrow(acc / sum);
 }

@@ -12,23 +12,7 @@
 
 #include <stdint.h>
 
-#include "pa_internal.h"
-
 namespace pa {
-
-// KV blocks the decode grid streams for sequence row (L keys, ql query rows,
-// skip shared blocks read by the cascade prefix pass): ceil(L / BS) - skip for
-// a decode row (ql == 1) whose lengths are in range, 0 for any other row, and
-// -1 for a decode row whose lengths are out of range (streamed as 0; the decode
-// grid raises PA_FLAG_CONTEXT_RANGE). The decode grids and the merge kernel
-// all count with this one rule.
-template <int BS>
-__device__ __forceinline__ int decode_blocks(int L, int ql, int skip, const DecodeArgs& a) {
-  if (ql != 1) return 0;
-  if (L < 1 || L > a.max_context_len || L > a.max_blocks_per_seq * BS || skip < 0 || skip > (L + BS - 1) / BS)
-    return -1;
-  return (L + BS - 1) / BS - skip;
-}
 
 // First CTA whose range [c*B/G, (c+1)*B/G) contains block b (0 <= b < B).
 __device__ __forceinline__ int cta_of_block(int64_t b, int64_t B, int G) {

@@ -190,11 +190,14 @@ __global__ void __launch_bounds__(192, 1)
       const int L = __ldg(a.context_lens + s);
       const int r0 = __ldg(a.query_start_loc + s);
       const int ql = __ldg(a.query_start_loc + s + 1) - r0;
-      const int skip = (ql == 1 && a.skip_blocks) ? __ldg(a.skip_blocks + s) : 0;
-      n = decode_blocks<BS>(L, ql, skip, a);
-      if (n < 0) {
-        raise_flag(a.status, PA_FLAG_CONTEXT_RANGE);
-        n = 0;
+      if (ql == 1) {
+        const int skip = a.skip_blocks ? __ldg(a.skip_blocks + s) : 0;
+        if (L < 1 || L > a.max_context_len || L > a.max_blocks_per_seq * BS || skip < 0 ||
+            skip > (L + BS - 1) / BS) {
+          raise_flag(a.status, PA_FLAG_CONTEXT_RANGE);
+        } else {
+          n = (L + BS - 1) / BS - skip;
+        }
       }
     }
     int total;
