@@ -295,8 +295,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     // Every lane arrives on kv_full asynchronously, when its copies have
     // landed; the MMA thread fences them for the tensor cores. The first K warp
     // also loads each segment's two Q tiles (TMA), after the segment's first K
-    // tile: the Q buffer frees only when the previous segment's last scores are
-    // done. (More gathering warps keep more copies in flight: each warp
+    // tile (the Q buffer frees only when the previous segment's last scores are
+    // done), or before it for the CTA's first segment. (More gathering warps keep more copies in flight: each warp
     // sustains only a few bytes per cycle.)
     const int kv = warp - kLoadWarp < kKWarps ? 0 : 1;          // 0: K, 1: V
     const int wi = kv ? warp - kLoadWarp - kKWarps : warp - kLoadWarp;  // warp within its set
@@ -309,6 +309,25 @@ __global__ void __launch_bounds__(kThreads, 1)
     bool ok = true;
     uint32_t kt = 0, nq = 0;  // key tiles and segments of this CTA so far
     uint32_t my_q = 0;        // 1 + the segment of the last Q load this warp issued (0: none)
+    // both Q tiles of segment nq, once the previous segment's scores are done
+    auto load_q = [&](const PSeg& g) {
+      bool r = true;
+      if (lane == 0) {
+        r = mbar_wait(q_empty, (nq & 1) ^ 1, a.status, a.wait_limit_ns);
+        if (r) {
+          mbar_arrive_expect_tx(q_full, 2 * C::kQTileB);
+#pragma unroll
+          for (int qi = 0; qi < 2; ++qi)
+#pragma unroll
+            for (int h = 0; h < C::kHalves; ++h)
+              tma_load_3d(smem + qi * C::kQTileB + h * 128 * 128, &qmap, q_full, h * 64, g.hg * GH,
+                          g.r0 + g.pt * C::kPairTok + qi * C::kTOK);
+        }
+      }
+      r = __shfl_sync(0xffffffffu, r, 0) != 0;
+      if (r) my_q = nq + 1;
+      return r;
+    };
     for (int64_t b = beg; b < end && ok;) {
       PSeg g;
       locate<GH>(b, beg, end, cta, prefix, S, HGp, a, g);
@@ -325,6 +344,11 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (lane == 0) ok = mbar_wait(&kv_empty[sl], ((n / NSL) & 1) ^ 1, a.status, a.wait_limit_ns);
         ok = __shfl_sync(0xffffffffu, ok, 0) != 0;
         if (!ok) break;
+        // the CTA's first Q tiles go out before its first key tile: nothing
+        // holds their buffer yet
+        if (warp == kLoadWarp && j == g.j_lo && nq == 0) {
+          if (!(ok = load_q(g))) break;
+        }
         const uint32_t dst = smem_u32(smem + C::kStageOff + sl * C::kKB) + dst_col;
         // the tile's 128 rows in groups of 8 (one block holds whole groups):
         // warp wi takes groups wi, wi + nw, ...
@@ -349,22 +373,8 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
         }
         cp_async_arrive(&kv_full[sl]);
-        if (warp == kLoadWarp && j == g.j_lo) {  // this segment's Q tiles
-          if (lane == 0) {
-            ok = mbar_wait(q_empty, (nq & 1) ^ 1, a.status, a.wait_limit_ns);
-            if (ok) {
-              mbar_arrive_expect_tx(q_full, 2 * C::kQTileB);
-#pragma unroll
-              for (int qi = 0; qi < 2; ++qi)
-#pragma unroll
-                for (int h = 0; h < C::kHalves; ++h)
-                  tma_load_3d(smem + qi * C::kQTileB + h * 128 * 128, &qmap, q_full, h * 64, hq0,
-                              g.r0 + g.pt * C::kPairTok + qi * C::kTOK);
-            }
-          }
-          ok = __shfl_sync(0xffffffffu, ok, 0) != 0;
-          if (!ok) break;
-          my_q = nq + 1;
+        if (warp == kLoadWarp && j == g.j_lo && nq > 0) {  // a later segment's Q tiles
+          if (!(ok = load_q(g))) break;
         }
       }
       ++nq;
