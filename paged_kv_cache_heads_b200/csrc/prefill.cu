@@ -22,11 +22,12 @@
 //    splits the whole range evenly (stream-K): CTA c takes units
 //    [c*T/G, (c+1)*T/G). A pair one CTA covers entirely is written straight to
 //    the output; otherwise each covering CTA leaves a partial
-//    (O / l, m + log2 l) per row and prefill_combine_kernel merges them.
-//  * Warp 9 loads both Q tiles of a segment with TMA. Warps 9 and 10 gather
-//    each key tile's K and V rows through the block table with 16-byte
-//    cp.async copies straight into the 128-byte swizzled layout of the MMA
-//    operands (a tensor-copy box per KV block and 64 columns would cost one
+//    (O / l, m + log2 l) per row, the CTA that starts the pair records which
+//    CTAs cover it, and prefill_combine_kernel merges them.
+//  * Warp 9 loads both Q tiles of a segment with TMA. Warps 9-12 gather each
+//    key tile's K rows and warps 13-15 its V rows through the block table with
+//    16-byte cp.async copies straight into the 128-byte swizzled layout of the
+//    MMA operands (a tensor-copy box per KV block and 64 columns would cost one
 //    serialised issue each), into a ring of K/V stages. Rows at or beyond L
 //    (the unfilled tail of the last block, blocks past the sequence) are
 //    filled with zeros, so stale bits there cannot reach the output.
@@ -212,8 +213,9 @@ __global__ void __launch_bounds__(kThreads, 1)
   if (warp >= kLoadWarp && lane == 0) tma_prefetch_desc(&qmap);
   // The merge grid chained after this one may be scheduled now: its CTAs take
   // SMs as this grid's CTAs exit and wait there for this whole grid to finish,
-  // so the merge starts without a launch gap. (Every CTA of this grid is
-  // resident before any CTA can pass this point in all of them.)
+  // so the merge starts without a launch gap. (The merge grid is launched only
+  // once every CTA of this grid has executed this, so none of its CTAs can
+  // take an SM that a CTA of this grid still waits for.)
   launch_dependents();
 
   // ---- key tiles of every prefill sequence, and their prefix. This grid is
