@@ -667,6 +667,36 @@ def workload_config(wl, world: int, l2_note: str):
             "parallelism": "dp%d (independent replicas)" % world, "l2": l2_note}
 
 
+PREFILL_SCALING = (4, 16, 64)  # chunks of 256 tokens in the prefill-only scaling sweep
+
+
+def prefill_scaling(bf16_peak: float, flush, reps: int = 10):
+    """Prefill-only calls of n 256-token chunks (the mixed batches' geometry:
+    32 q / 8 kv heads, D 128, bf16, block size 16; prior contexts drawn from
+    U{0..1792}, seeded), the L2 flushed before each call: how the prefill rate
+    grows once the per-CTA fixed costs are spread over more key tiles."""
+    import numpy as np
+    import torch
+    from paged_kv_cache_heads_b200 import scenario as gs, workloads as W
+    out = {}
+    for n in PREFILL_SCALING:
+        ctx = [int(x) for x in np.random.default_rng(7 + n).integers(0, 1793, size=n)]
+        wl = W.random_case(900 + n, num_seqs=n, q_lens=[256] * n, ctx_extra=ctx, num_kv_heads=8, group=4,
+                           head_dim=128, block_size=16, dtype=W.BF16)
+        b = gs.prepare(wl)
+        gs.run_step(b)
+        torch.cuda.synchronize()
+        flops = sum(4 * 128 * 32 * (256 * c + 256 * 257 // 2) for c in ctx)
+        t = timed_calls(lambda: gs.run_attention(b), reps, flush)
+        ms = t["median_ms"]
+        out["chunks_%d" % n] = {"us": ms * 1e3, "gflop": flops / 1e9, "tflops": flops / ms / 1e9,
+                                "frac_of_bf16_peak": flops / ms / 1e9 / bf16_peak}
+        del b
+        torch.cuda.empty_cache()
+    out["l2"] = "flushed before each call (%d MB write, then %d MB read)" % (L2_FLUSH_BYTES >> 20, L2_FLUSH_BYTES >> 20)
+    return out
+
+
 def build_workload(name: str):
     from paged_kv_cache_heads_b200 import workloads as W
     if name == "prefix_cow_p2000":
@@ -747,6 +777,7 @@ def main():
             for name in SWEEP:
                 configs[name] = measure_config(name, hbm_peak, bf16_peak, flush,
                                                oracle=not args.no_cpu_baseline)
+            configs["prefill_scaling"] = prefill_scaling(bf16_peak, flush)
         configs["clocks"] = sweep_clocks.summary()
         del flush
 
