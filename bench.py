@@ -191,6 +191,14 @@ def barrier():
 # algorithmic work of one step
 # --------------------------------------------------------------------------
 
+def causal_prefill_flops(L: int, ql: int, head_dim: int, num_q_heads: int) -> int:
+    """FLOPs of the prefill rows of one sequence: query row j (absolute
+    position L - ql + j) sees L - ql + j + 1 keys, and each (row, key) pair
+    costs 2 * head_dim for Q.K and 2 * head_dim for P.V, per query head."""
+    pairs = ql * (L - ql) + ql * (ql + 1) // 2   # = sum over j < ql of (L - ql + j + 1)
+    return 4 * head_dim * num_q_heads * pairs
+
+
 def step_work(wl, step_tokens: int, step_pairs: int):
     """Algorithmic bytes / flops of one step, from the workload's sizes only."""
     geo = wl.geometry
@@ -204,8 +212,7 @@ def step_work(wl, step_tokens: int, step_pairs: int):
         attn_kv += 2 * L * row + 4 * ((L + geo.block_size - 1) // geo.block_size)
         attn_qo += 2 * ql * geo.num_q_heads * geo.head_dim * e
         if ql > 1:
-            pairs = sum(L - ql + j + 1 for j in range(ql))
-            prefill_flops += 4 * geo.head_dim * pairs * geo.num_q_heads
+            prefill_flops += causal_prefill_flops(L, ql, geo.head_dim, geo.num_q_heads)
     store = 2 * 2 * step_tokens * row + 4 * step_tokens
     copy = 2 * 2 * step_pairs * geo.block_size * row
     return dict(attn_bytes=attn_kv + attn_qo, attn_kv_bytes=attn_kv, store_bytes=store, copy_bytes=copy,
@@ -532,7 +539,7 @@ def prefill_only_call(b):
     flops = 0
     for i in pre:
         L, ql = int(lens[i]), wl.q_lens[i]
-        flops += 4 * geo.head_dim * geo.num_q_heads * sum(L - ql + j + 1 for j in range(ql))
+        flops += causal_prefill_flops(L, ql, geo.head_dim, geo.num_q_heads)
 
     def fn():
         P.pa_attention(b.q, b.k_cache, b.v_cache, bt, geo.max_blocks_per_seq, cl, qs, len(pre), t,
@@ -686,7 +693,7 @@ def prefill_scaling(bf16_peak: float, flush, reps: int = 10):
         b = gs.prepare(wl)
         gs.run_step(b)
         torch.cuda.synchronize()
-        flops = sum(4 * 128 * 32 * (256 * c + 256 * 257 // 2) for c in ctx)
+        flops = sum(causal_prefill_flops(c + 256, 256, 128, 32) for c in ctx)
         t = timed_calls(lambda: gs.run_attention(b), reps, flush)
         ms = t["median_ms"]
         out["chunks_%d" % n] = {"us": ms * 1e3, "gflop": flops / 1e9, "tflops": flops / ms / 1e9,

@@ -68,3 +68,20 @@ def test_reference_arm_line_on_rank0():
     line = json.loads(r.stdout.strip().splitlines()[-1])
     assert line["impl"] == "reference" and line["unit"] == "query-tokens/s" and line["value"] > 0
     assert line["e2e"]["h2d_bytes_per_step"] == 0 and line["cpu_baseline"]["kind"] == "oracle"
+
+
+def test_causal_prefill_flops_counts_every_visible_key():
+    """The FLOP count behind the prefill TFLOP/s figures: against a count of
+    (query row, visible key) pairs enumerated one by one."""
+    import random
+    import bench
+    rng = random.Random(5)
+    for _ in range(20):
+        ql = rng.randint(1, 300)
+        L = ql + rng.randint(0, 2000)
+        d, h = rng.choice([64, 128]), rng.choice([1, 8, 32])
+        pairs = 0
+        for j in range(ql):
+            pos = L - ql + j
+            pairs += sum(1 for key in range(L) if key <= pos)
+        assert bench.causal_prefill_flops(L, ql, d, h) == 4 * d * h * pairs
